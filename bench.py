@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark of the Llama-3-8B-shape decoder on B200: prefill + greedy decode tokens/s.
+
+One step = the whole hot path over one batch of the workload
+"llama3-8b-bf16-b1-p2048-g256": prefill of a 2048-token prompt (batch 1), then
+256 greedy decode steps feeding back the argmax, on seeded random bf16 weights
+of the Llama-3-8B architecture (32 layers, dim 4096, 32/8 heads, FFN 14336,
+vocab 128256). Inputs are resident in HBM when the timed region starts.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 run under torch.distributed.run: every rank runs an independent
+replica on its own GPU (the decoder has no exchange step), times are the max
+over ranks, and value is the tokens of all ranks / that time.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "llama3-8b-bf16-b1-p2048-g256"
+METRIC = "decode & prefill tokens/s at Llama-3-8B shape, 1 B200; % of HBM/tensor roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ---------------------------------------------------------------- algorithmic work
+def work_model(shape, B, T, S_decode_mean):
+    """Algorithmic FLOPs of the prefill and bytes of one decode step."""
+    D, H, Hk, d, F, V, L = (shape.dim, shape.n_heads, shape.n_kv_heads, shape.head_dim, shape.ffn_hidden,
+                            shape.vocab, shape.n_layers)
+    lin_params = L * (D * (H + 2 * Hk) * d + H * d * D + 3 * D * F)
+    prefill_flops = 2 * B * T * lin_params + L * B * (4 * H * d * T * T / 2) + 2 * B * D * V
+    w_bytes = 2 * (lin_params + V * D)
+    kv_bytes = L * B * 2 * Hk * d * 2 * S_decode_mean
+    kinds_bytes = {  # one decode launch, B rows
+        "qkv": 2 * D * (H + 2 * Hk) * d, "wo": 2 * H * d * D, "w13": 2 * 2 * F * D, "w2": 2 * F * D,
+        "head": 2 * V * D, "attn": B * 2 * Hk * d * 2 * S_decode_mean,
+    }
+    kinds_flops = {"qkv": 2 * B * T * D * (H + 2 * Hk) * d, "wo": 2 * B * T * H * d * D, "w13": 2 * B * T * 2 * F * D,
+                   "w2": 2 * B * T * F * D, "attn": B * 4 * H * d * T * T / 2}
+    return prefill_flops, w_bytes + kv_bytes, kinds_bytes, kinds_flops
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 9 and f[1].replace(".", "").isdigit():
+                    rows.append(f)
+        except Exception:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm = [float(r[1]) for r in rows]
+        smax = float(rows[0][2])
+        loaded = [s for s, r in zip(sm, rows) if float(r[3] or 0) > 300] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3] or 0) for r in rows)}
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+def oracle_sample(shape, seed, prompt_len, decode_steps, budget_s=20.0):
+    """Time the fp64 oracle on one decoder layer of the workload and extrapolate.
+
+    Sample: layer 0 at full width; a prefill of Ts prompt tokens and a decode step
+    against a cache of prompt_len positions; the lm_head on a vocab slice. The
+    whole-step time is estimated as n_layers * (prompt_len * t_prefill_token +
+    decode_steps * t_decode) + (decode_steps + 1) * t_head. Attention cost of the
+    full prompt is underestimated by timing a shorter prefill (stated in `sample`).
+    """
+    import numpy as np
+    import torch
+    import oracle as O
+    import seeded_inputs as S
+    t0 = time.time()
+    one = shape.replace(n_layers=1, has_embed_and_head=False)
+    lw = S.make_layer_weights(one, seed, 0)
+    orc = O.OracleModel(one, {}, [lw], batch=1)
+    orc.layer(0)  # widen the layer's weights once (not timed)
+    Ts = 512
+    h = S.make_hidden(seed, 1, Ts, shape.dim, tag="oracle-sample").numpy()
+    t = time.perf_counter()
+    orc.forward_hidden(h)
+    t_prefill_tok = (time.perf_counter() - t) / Ts
+    # decode against a prompt_len cache
+    g = np.random.default_rng(0)
+    orc.set_cache(0, 0, g.standard_normal((prompt_len, shape.n_kv_heads, shape.head_dim)),
+                  g.standard_normal((prompt_len, shape.n_kv_heads, shape.head_dim)))
+    n_dec = 0
+    t = time.perf_counter()
+    while n_dec < 10 and time.perf_counter() - t < budget_s / 2:
+        orc.forward_hidden(h[:, :1])
+        n_dec += 1
+    t_decode = (time.perf_counter() - t) / n_dec
+    rows = 8192
+    Wslice = np.random.default_rng(1).standard_normal((rows, shape.dim))
+    x = np.random.default_rng(2).standard_normal(shape.dim)
+    t = time.perf_counter()
+    O.argmax_first(x @ Wslice.T)
+    t_head = (time.perf_counter() - t) * shape.vocab / rows
+    est = shape.n_layers * (prompt_len * t_prefill_tok + decode_steps * t_decode) + (decode_steps + 1) * t_head
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=os.cpu_count())
+    except Exception:
+        cores = os.cpu_count()
+    return {
+        "value": (prompt_len + decode_steps) / est, "unit": "tokens/s", "cores": int(cores), "kind": "oracle",
+        "sample": (f"fp64 oracle, layer 0 of 32 at full width: prefill of {Ts} tokens and {n_dec} decode "
+                   f"steps against a {prompt_len}-position cache, lm_head on {rows} of {shape.vocab} rows; "
+                   f"extrapolated to the full step ({prompt_len} prefill + {decode_steps} decode tokens, "
+                   f"{shape.n_layers} layers; prefill attention of the full prompt underestimated)"),
+        "estimated_step_s": est, "wall_s": time.time() - t0,
+    }
+
+
+def run_reference(args, rank):
+    """--impl reference: the CPU oracle as it stands, on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    import seeded_inputs as S
+    w = S.WORKLOADS[WORKLOAD]
+    vals = []
+    last = None
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample(w.shape, w.seed, w.prompt_len, w.decode_steps, budget_s=8.0)
+        if i >= args.warmup:
+            vals.append(r["value"])
+        last = r
+    v = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * (w.prompt_len + w.decode_steps) / v,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,0.02) weights, N(0,1) hidden states)",
+            "config": {"workload": WORKLOAD, "batch": w.batch, "prompt_len": w.prompt_len,
+                       "decode_steps": w.decode_steps},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": last["cores"], "kind": "oracle",
+                             "sample": last["sample"]},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- ncu traffic record
+def ncu_traffic(kind):
+    """DRAM bytes per launch of a kernel kind from the committed ncu summary, if it is current."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(kind)
+    if not rec:
+        return None
+    src = open(os.path.join(ROOT, "llama_decoder_forward_fwd_b200", "csrc", rec["source"]), "rb").read()
+    if hashlib.sha256(src).hexdigest()[:16] != rec["source_sha"]:
+        return None  # the kernel changed since the counters were taken
+    return rec["dram_bytes_per_launch"]
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import llama_decoder_forward_fwd_b200 as L
+    import seeded_inputs as S
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = S.WORKLOADS[WORKLOAD]
+    shape, B, T, G = w.shape, w.batch, w.prompt_len, w.decode_steps
+    peaks, peak_src = load_peaks()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+        cpu = oracle_sample(shape, w.seed, T, G)  # before the first GPU call
+
+    glob, layers = S.make_weights(shape, w.seed, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    model = L.Model(shape, glob, layers, max_batch=B, max_tokens=B * T,
+                    flags=0 if args.no_graph else L.LLM_FLAG_CUDA_GRAPH, stream=stream, device=dev)
+    prompt = S.make_tokens(w.seed, B, T, shape.vocab).to(dev)
+    gen = torch.zeros(G + 1, B, dtype=torch.int32, device=dev)
+
+    def one_step(ev=None):
+        L.llm_kv_cache_reset(model.h)
+        L.llm_prefill(model.h, prompt, gen[0])
+        if ev is not None:
+            ev.record(stream)
+        for i in range(G):
+            L.llm_decode_step(model.h, gen[i], gen[i + 1])
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize(dev)
+
+    # ---- timed region (device time, CUDA events on the model's stream) ----
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clk:
+        for k in range(args.steps):
+            starts[k].record(stream)
+            one_step(mids[k])
+            ends[k].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    pre_ms = [s.elapsed_time(m) for s, m in zip(starts, mids)]
+    dec_ms = [m.elapsed_time(e) for m, e in zip(mids, ends)]
+    total_s = max_over_ranks(sum(step_ms) / 1e3)
+    clocks = clk.summary()
+    L.llm_synchronize(model.h)
+    tokens_per_step = B * (T + G)
+    value = world * args.steps * tokens_per_step / total_s
+
+    S_mean = T + G / 2
+    prefill_flops, decode_bytes, kbytes, kflops = work_model(shape, B, T, S_mean)
+    pre_s = max_over_ranks(statistics.mean(pre_ms) / 1e3)
+    dec_s = max_over_ranks(statistics.mean(dec_ms) / 1e3)
+    prefill = {"tok_s": B * T / pre_s, "ms": pre_s * 1e3, "tflops": prefill_flops / pre_s / 1e12,
+               "frac_of_bf16_peak": prefill_flops / pre_s / 1e12 / peaks["bf16_tflops"],
+               "peak_tflops": peaks["bf16_tflops"], "peak_kind": f"{peak_src} burst"}
+    decode = {"tok_s": B * G / dec_s, "ms_per_token": dec_s * 1e3 / G,
+              "gbs": decode_bytes * G / dec_s / 1e9,
+              "frac_of_hbm": decode_bytes * G / dec_s / 1e9 / peaks["hbm_gbs"], "peak_gbs": peaks["hbm_gbs"],
+              "bytes_per_step": decode_bytes}
+
+    # ---- e2e: host buffers through the public API, copies inside the timed region ----
+    host_prompt = prompt.cpu().pin_memory()
+    host_out = torch.empty_like(gen, device="cpu").pin_memory()
+    dprompt = torch.empty_like(prompt)
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    for k in range(args.steps):
+        e_s[k].record(stream)
+        with torch.cuda.stream(stream):
+            dprompt.copy_(host_prompt, non_blocking=True)
+        L.llm_kv_cache_reset(model.h)
+        L.llm_prefill(model.h, dprompt, gen[0])
+        for i in range(G):
+            L.llm_decode_step(model.h, gen[i], gen[i + 1])
+        with torch.cuda.stream(stream):
+            host_out.copy_(gen, non_blocking=True)
+        e_e[k].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_s = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)) / 1e3)
+    e2e = {"value": world * args.steps * tokens_per_step / e2e_s, "unit": "tokens/s",
+           "h2d_bytes_per_step": host_prompt.numel() * 4, "d2h_bytes_per_step": host_out.numel() * 4}
+
+    # ---- per-kernel CUDA-event timing of one step (roofline of the dominant kernel) ----
+    tm = L.Model(shape, model.glob, model.layers, max_batch=B, max_tokens=B * T,
+                 flags=L.LLM_FLAG_KERNEL_TIMING, stream=stream, device=dev)
+    gen2 = torch.zeros_like(gen)
+    L.llm_prefill(tm.h, prompt, gen2[0])
+    kt_pre = L.llm_kernel_times(tm.h, reset=True)
+    for i in range(G):
+        L.llm_decode_step(tm.h, gen2[i], gen2[i + 1])
+    kt_dec = L.llm_kernel_times(tm.h, reset=True)
+    tm.free()
+    shares = {}
+    for name, (ms, n) in kt_pre.items():
+        if n:
+            shares["prefill/" + name] = (ms, n)
+    for name, (ms, n) in kt_dec.items():
+        if n:
+            shares["decode/" + name] = (ms, n)
+    tot = sum(ms for ms, _ in shares.values())
+    dom = max(shares, key=lambda k: shares[k][0])
+    ms, n = shares[dom]
+    avg_s = ms / n / 1e3
+    phase, kind = dom.split("/")
+    if phase == "decode" and kind in kbytes:
+        achieved = kbytes[kind] / avg_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": ncu_traffic("decode/" + kind),
+                "kernel": dom, "bytes_per_launch": kbytes[kind], "avg_launch_us": avg_s * 1e6,
+                "launches": n, "peak_source": f"{peak_src} hbm_gbs"}
+    else:
+        per = kflops.get(kind, 0)
+        achieved = per / avg_s / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": ncu_traffic(dom), "kernel": dom,
+                "flops_per_launch": per, "avg_launch_us": avg_s * 1e6, "launches": n,
+                "peak_source": f"{peak_src} bf16_tflops (burst)"}
+    kernel_table = {k: {"ms": round(v[0], 3), "launches": v[1], "share": round(v[0] / tot, 4)}
+                    for k, v in sorted(shares.items(), key=lambda kv: -kv[1][0])}
+    model.free()
+
+    if rank != 0:
+        return
+    line = {
+        "impl": "ours", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_s * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,0.02) bf16 weights of the Llama-3-8B architecture, uniform token ids",
+        "config": {"workload": WORKLOAD, "batch": B, "prompt_len": T, "decode_steps": G,
+                   "layers": shape.n_layers, "dim": shape.dim, "vocab": shape.vocab,
+                   "l2": "inputs larger than L2: every step streams 16 GB of weights",
+                   "cuda_graph_decode": not args.no_graph, "parallelism": f"replicas x{world}"},
+        "prefill": prefill, "decode": decode, "roofline": roof, "kernels": kernel_table,
+        "cpu_baseline": ({k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")} if cpu else None),
+        "e2e": e2e,
+        "gpu_launches": args.steps * (G + 1) * (5 * shape.n_layers + 2),
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,254 @@
+/*
+ * llama_fwd.h: C ABI of a Llama-2/3 decoder forward pass (prefill plus
+ * KV-cached greedy decode) on one NVIDIA B200 (sm_100a).
+ *
+ * What the calls compute. The pages this library follows define the
+ * decoder step by step, and every call below names its source by page title and
+ * section:
+ *   - "Building llama3 from scratch": params.json fields (the config struct), the
+ *     checkpoint tensor names and [out, in] shapes (the weights struct), the
+ *     embedding lookup, the RMSNorm code block, the per-head view of wq.
+ *   - "Model Llama 3 yang Diimplementasikan dengan NumPy Murni" (llama3.np):
+ *     "RoPE #1/#2", "QKV", "KV cache", "GQA", "Scaled Dot-Product Attention",
+ *     "Feed Forward", "Linear" (last-position logits), "Generasi" (prefill and
+ *     decode phases).
+ *   - "Resumen de una implementación desde cero del modelo LLaMA-3": attention
+ *     with a future-token mask and softmax, multi-head concat, SwiGLU, residuals,
+ *     final RMSNorm, logits, argmax as the next token.
+ *
+ * Conventions for every call:
+ *   - Pointers marked "device" are CUDA device pointers on the model's device;
+ *     "host" pointers are ordinary CPU memory.
+ *   - Matrices are row-major. Weight matrices are [out, in]: y = x W^T.
+ *   - Work is queued on the model's CUDA stream and is asynchronous: device
+ *     outputs are valid after llm_synchronize() or a sync of that stream.
+ *   - Every int-returning call returns LLM_OK (0) or a negative LLM_ERR_* code
+ *     and never aborts the process. llm_last_error() gives a message for the
+ *     last failure on the calling thread.
+ *   - Argument errors (null pointers, sizes beyond the limits given at init,
+ *     unsupported shapes) are detected on the host before anything is queued.
+ *   - Device-side waits are bounded; a wait that runs out sets the model's
+ *     error word, which llm_synchronize() reports as LLM_ERR_DEVICE_TIMEOUT.
+ */
+#ifndef LLAMA_FWD_H
+#define LLAMA_FWD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define LLM_OK                   0
+#define LLM_ERR_BAD_CONFIG      (-1)  /* inconsistent or unsupported config */
+#define LLM_ERR_NULL_PTR        (-2)  /* a required pointer is NULL */
+#define LLM_ERR_SEQ_OVERFLOW    (-3)  /* cache length + new tokens > max_seq_len */
+#define LLM_ERR_BATCH           (-4)  /* B < 1, B > max_batch, or B*T > max_tokens */
+#define LLM_ERR_CUDA            (-5)  /* a CUDA runtime/driver call failed */
+#define LLM_ERR_DEVICE_TIMEOUT  (-6)  /* a bounded device-side wait ran out */
+#define LLM_ERR_UNSUPPORTED     (-7)  /* valid request this build does not implement */
+#define LLM_ERR_BAD_ARG         (-8)  /* other invalid argument (e.g. a size) */
+
+/* ---- element types ----------------------------------------------------- */
+#define LLM_F32   0   /* weights, activations and KV cache in fp32 */
+#define LLM_BF16  1   /* bf16 weights/activations/KV cache, fp32 accumulation
+                         and fp32 residual stream */
+
+/* ---- config flags ------------------------------------------------------ */
+#define LLM_FLAG_CUDA_GRAPH  1  /* replay decode steps from captured CUDA graphs */
+#define LLM_FLAG_DEBUG_TAPS  2  /* keep each layer's output hidden state (see llm_debug_tap) */
+#define LLM_FLAG_KERNEL_TIMING 4 /* time every launch with CUDA events (see llm_kernel_times);
+                                    ignored for graph-replayed decode steps */
+
+/* ---- kernel kinds reported by llm_kernel_times ------------------------- */
+#define LLM_K_EMBED    0   /* embedding lookup / hidden-state load */
+#define LLM_K_QKV      1   /* QKV projection + RoPE + KV-cache append */
+#define LLM_K_ATTN     2   /* attention (flash or split-KV) */
+#define LLM_K_WO       3   /* wo projection + residual */
+#define LLM_K_W13      4   /* w1/w3 projection + SwiGLU */
+#define LLM_K_W2       5   /* w2 projection + residual */
+#define LLM_K_HEAD     6   /* final norm + lm_head + argmax */
+#define LLM_K_OUT      7   /* hidden-state output */
+#define LLM_K_COUNT    8
+
+/*
+ * Model hyper-parameters: the params.json fields of "Building llama3 from
+ * scratch" (dim, n_layers, n_heads, n_kv_heads, vocab_size, norm_eps, rope_theta),
+ * plus the FFN hidden size given explicitly and the capacity limits.
+ *   head_dim       must equal dim / n_heads; n_heads % n_kv_heads == 0.
+ *   max_seq_len    KV-cache positions per sequence.
+ *   max_batch      sequences (B) per call.
+ *   max_tokens     B*T per prefill call (0 means max_batch * max_seq_len).
+ *   dtype          LLM_F32 or LLM_BF16 (type of every weight buffer).
+ *   tie_embeddings lm_head reuses tok_emb (weights.out ignored).
+ *   has_embed_and_head  0 for a bare layer stack driven by the *_hidden calls.
+ */
+typedef struct llm_config {
+    int dim, n_layers, n_heads, n_kv_heads, head_dim, ffn_hidden, vocab;
+    int max_seq_len, max_batch, max_tokens;
+    float norm_eps, rope_theta;
+    int dtype;
+    int tie_embeddings;
+    int has_embed_and_head;
+    int flags;
+} llm_config;
+
+/*
+ * Weights: device pointers of element type config.dtype, owned by the caller,
+ * which must keep them alive and unchanged until llm_model_free(). Names follow
+ * the checkpoint keys listed in "Building llama3 from scratch". Per-layer
+ * fields are host arrays of n_layers device pointers (copied at init).
+ *   tok_emb    [vocab, dim]          (NULL when has_embed_and_head == 0)
+ *   out        [vocab, dim]          lm_head; NULL when tied
+ *   final_norm [dim]
+ *   attn_norm, ffn_norm [dim]
+ *   wq [n_heads*head_dim, dim], wk/wv [n_kv_heads*head_dim, dim],
+ *   wo [dim, n_heads*head_dim], w1/w3 [ffn_hidden, dim], w2 [dim, ffn_hidden]
+ * Every device pointer must be 16-byte aligned.
+ */
+typedef struct llm_weights {
+    const void *tok_emb, *out, *final_norm;
+    const void *const *attn_norm, *const *wq, *const *wk, *const *wv, *const *wo;
+    const void *const *ffn_norm, *const *w1, *const *w3, *const *w2;
+} llm_weights;
+
+typedef struct llm_model llm_model;
+
+/*
+ * Create a model on the current CUDA device. stream is a cudaStream_t on which
+ * every later call queues its work; NULL makes the model create and own a
+ * blocking stream (ordered with the legacy default stream) instead. The
+ * library allocates and owns the KV cache [n_layers][max_batch][n_kv_heads]
+ * [max_seq_len][head_dim] (element type dtype), the RoPE cos/sin tables, the
+ * activations and the scratch; llm_model_free() releases them. All cache
+ * lengths start at 0. On failure *out is NULL.
+ */
+int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, llm_model** out);
+
+/*
+ * Prefill phase ("Generasi": the whole prompt at once). tokens: device int32
+ * [B, T]. Sequence b's tokens take positions len[b] .. len[b]+T-1, where len[b]
+ * is its current cache length (0 after init/reset); their K and V are appended to
+ * the cache and len[b] grows by T. Writes next[b] (device int32 [B]) = argmax of
+ * the logits at the last position (ties: lowest id), and, when logits is not
+ * NULL, those logits (device fp32 [B, vocab]).
+ * Errors: NULL_PTR, BATCH, SEQ_OVERFLOW, BAD_CONFIG (model built without
+ * embedding/head).
+ */
+int llm_prefill(llm_model* m, const int32_t* tokens, int B, int T, int32_t* next, float* logits);
+
+/*
+ * Prefill of the layer stack on given hidden states, with no embedding, final
+ * norm or lm_head. h_in: device fp32 [B, T, dim]; h_out: device fp32 [B, T, dim],
+ * the last layer's output. Positions and cache growth as in llm_prefill.
+ */
+int llm_prefill_hidden(llm_model* m, const float* h_in, int B, int T, float* h_out);
+
+/*
+ * One decode step ("KV cache": only the newest token is projected; "Generasi":
+ * decode phase). in_tok: device int32 [B], the token at position len[b] of
+ * sequence b; next: device int32 [B], the greedy next token; logits: optional
+ * device fp32 [B, vocab]. Grows len[b] by 1. B may differ from the last
+ * prefill's B; sequences b < B are advanced.
+ */
+int llm_decode_step(llm_model* m, int B, const int32_t* in_tok, int32_t* next, float* logits);
+
+/* As llm_decode_step, on hidden states: h_in, h_out device fp32 [B, dim]. */
+int llm_decode_step_hidden(llm_model* m, int B, const float* h_in, float* h_out);
+
+/* Set every sequence's cache length to 0 (cache contents are left in place). */
+int llm_kv_cache_reset(llm_model* m);
+
+/*
+ * Direct access to the cache for callers that fill it themselves. *k and *v get
+ * the device base pointers of K and V (element type dtype; entries hold
+ * post-RoPE keys and plain values). strides[0..3] get the element strides of
+ * [layer, batch, kv_head, position]; head_dim is contiguous. The memory stays
+ * owned by the model.
+ */
+int llm_kv_cache_view(llm_model* m, void** k, void** v, int64_t strides[4]);
+
+/* Set (host int32 [B]) or read back the cache lengths of sequences 0..B-1. */
+int llm_kv_cache_set_lens(llm_model* m, const int32_t* lens, int B);
+int llm_kv_cache_get_lens(llm_model* m, int32_t* lens, int B);
+
+/*
+ * Copy the output hidden state of decoder layer `layer` (fp32 residual stream,
+ * [tokens, dim] with tokens = B*T of the last prefill or B of the last decode
+ * step) into dst (device fp32, dst_elems elements at least). Needs
+ * LLM_FLAG_DEBUG_TAPS at init.
+ */
+int llm_debug_tap(llm_model* m, int layer, float* dst, size_t dst_elems);
+
+/*
+ * Per-kind kernel time recorded since the last reset (LLM_FLAG_KERNEL_TIMING).
+ * Synchronises the stream, then writes total milliseconds and launch counts of
+ * kinds 0..n-1 (see LLM_K_*) into the host arrays total_ms[n] and launches[n];
+ * reset != 0 clears the record afterwards. Kernels are timed with a CUDA event
+ * pair each on the model's stream, so kernels that would otherwise overlap
+ * their neighbours' tails run back to back while timing is on.
+ */
+int llm_kernel_times(llm_model* m, int n, double* total_ms, int64_t* launches, int reset);
+
+/* Wait for the model's stream; report a CUDA error or a device-side timeout. */
+int llm_synchronize(llm_model* m);
+
+/* Release everything the model allocated. NULL is accepted. */
+void llm_model_free(llm_model* m);
+
+/* Message describing the last failure on this thread ("" if none). */
+const char* llm_last_error(void);
+
+/* ======================================================================
+ * Single-operation entry points. Each runs one of the model's kernels on
+ * caller-provided device buffers, on `stream` (a cudaStream_t, NULL: default).
+ * ==================================================================== */
+
+/*
+ * C = A B^T on the tensor cores (the prefill projection kernel, tcgen05/TMEM
+ * fed by TMA). A: device bf16 [M, K]; B: device bf16 [N, K]; C: device fp32
+ * [M, N]. fp32 accumulation. Needs K % 64 == 0, N % 256 == 0, 16-byte aligned
+ * pointers; M >= 1 is arbitrary. Source: "Building llama3 from scratch", the
+ * projection q_per_token = x @ wq_head^T, here for whole matrices.
+ */
+int llm_op_gemm_bf16(const void* A, const void* B, float* C, int M, int N, int K, void* stream);
+
+/*
+ * y = x W^T for a few rows (the decode projection kernel). x: device bf16
+ * [M, K] with M <= 16; W: device bf16 [N, K]; y: device fp32 [M, N].
+ * Needs K % 8 == 0.
+ */
+int llm_op_gemv_bf16(const void* x, const void* W, float* y, int M, int N, int K, void* stream);
+
+/*
+ * Causal grouped-query attention over a KV cache for a block of new tokens
+ * ("Implementación de la atención" and "Atención multi-head" in "Resumen ...";
+ * "GQA" and "Scaled Dot-Product Attention" in llama3.np).
+ *   q:      device [B, T, H, d], element type dtype, RoPE already applied
+ *   kcache, vcache: device [B, Hk, S_max, d] (one layer's cache), dtype
+ *   pos0:   device int32 [B]; query t of sequence b sits at position pos0[b]+t
+ *           and attends to keys 0 .. pos0[b]+t of its sequence
+ *   out:    device [B, T, H*d], dtype
+ * Scale 1/sqrt(d); query head h reads KV head h / (H/Hk).
+ * llm_op_attention_prefill is the flash (tensor-core) kernel: dtype LLM_BF16,
+ * d == 128. llm_op_attention_decode is the split-KV kernel: any dtype,
+ * d <= 128 with d % 8 == 0, H/Hk*T <= 16; it needs a device scratch buffer of
+ * llm_op_attention_decode_workspace(...) bytes (16-byte aligned, contents
+ * arbitrary; the kernel leaves it ready for the next call, so calls sharing one
+ * buffer must not overlap in time).
+ */
+int llm_op_attention_prefill(const void* q, const void* kcache, const void* vcache,
+                             const int32_t* pos0, void* out, int B, int T, int H, int Hk,
+                             int d, int S_max, int dtype, void* stream);
+size_t llm_op_attention_decode_workspace(int B, int T, int H, int Hk, int d);
+int llm_op_attention_decode(const void* q, const void* kcache, const void* vcache,
+                            const int32_t* pos0, void* out, int B, int T, int H, int Hk,
+                            int d, int S_max, int dtype, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LLAMA_FWD_H */

@@ -1,0 +1,295 @@
+// Prefill projections on the 5th-generation tensor cores: C = A W^T with
+// A = activations [M][K] bf16 and W = a weight matrix [N][K] bf16 ("Building
+// llama3 from scratch": q_per_token = x @ wq_head^T, here for all tokens and all
+// heads at once), fp32 accumulation in tensor memory.
+//
+// Persistent kernel, one CTA per SM, 6 warps:
+//   warp 0     TMA producer: streams 128x64 A tiles and 256x64 B tiles into a
+//              4-stage shared-memory ring (128-byte swizzle), one mbarrier per
+//              stage for "full" (transaction bytes) and one for "empty".
+//   warp 1     allocates 512 TMEM columns and issues tcgen05.mma (M=128, N=256,
+//              K=16; four per 64-wide k block) from one elected thread into one
+//              of two 256-column accumulators, committing "empty" per stage and
+//              "accumulator full" per tile.
+//   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter (rows) of the
+//              accumulator, the fused epilogue (RMSNorm scale, RoPE + KV-cache
+//              append, SwiGLU, or residual add) and stores; then release the
+//              accumulator so the MMA warp can start the tile after next.
+// Tiles are visited m-fastest so CTAs running together share weight tiles in L2.
+#include "epilogue.cuh"
+
+namespace lfw {
+
+constexpr int G_STAGES = 4;
+constexpr int G_A_BYTES = GEMM_BM * GEMM_BK * 2;  // 16 KB
+constexpr int G_B_BYTES = GEMM_BN * GEMM_BK * 2;  // 32 KB
+constexpr int G_STAGE_BYTES = G_A_BYTES + G_B_BYTES;
+constexpr int G_SMEM_BYTES = G_STAGES * G_STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int G_THREADS = 192;
+constexpr uint32_t G_TMEM_COLS = 512;
+
+struct GemmKernelParams {
+    int seg_cols[3];
+    int M, N, K;
+    Epi epi;
+};
+
+template <int EPI>
+__global__ void __launch_bounds__(G_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                   const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
+                   const GemmKernelParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + G_STAGES * G_STAGE_BYTES);
+    uint64_t* empty = full + G_STAGES;
+    uint64_t* tfull = empty + G_STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t* err = p.epi.err;
+
+    if (warp == 0 && lane == 0) {
+        for (int i = 0; i < G_STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], 4);
+        }
+        fence_mbar_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB0);
+        tma_prefetch_desc(&tmB1);
+        tma_prefetch_desc(&tmB2);
+    }
+    if (warp == 1) {
+        tc_alloc(tmem_slot, G_TMEM_COLS);
+        tc_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    pdl_trigger();
+    pdl_wait();
+
+    const int num_m = (p.M + GEMM_BM - 1) / GEMM_BM;
+    const int num_n = (EPI == EPI_SWIGLU) ? p.N / (GEMM_BN / 2) : p.N / GEMM_BN;
+    const int total = num_m * num_n;
+    const int nk = p.K / GEMM_BK;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const int mb = tile % num_m, nb = tile / num_m;
+                const CUtensorMap* b0;
+                const CUtensorMap* b1;
+                int r0, r1;
+                if (EPI == EPI_SWIGLU) {
+                    b0 = &tmB0;
+                    b1 = &tmB1;
+                    r0 = r1 = nb * (GEMM_BN / 2);
+                } else {
+                    int c = nb * GEMM_BN, s = 0;
+                    while (s < 2 && c >= p.seg_cols[s]) {
+                        c -= p.seg_cols[s];
+                        ++s;
+                    }
+                    b0 = b1 = (s == 0) ? &tmB0 : (s == 1) ? &tmB1 : &tmB2;
+                    r0 = c;
+                    r1 = c + GEMM_BN / 2;
+                }
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, err, DERR_GEMM_PRODUCER_WAIT)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + stage * G_STAGE_BYTES;
+                    uint8_t* sb = sa + G_A_BYTES;
+                    mbar_arrive_expect_tx(&full[stage], G_STAGE_BYTES);
+                    tma_load_2d(sa, &tmA, &full[stage], kb * GEMM_BK, mb * GEMM_BM);
+                    tma_load_2d(sb, b0, &full[stage], kb * GEMM_BK, r0);
+                    tma_load_2d(sb + G_B_BYTES / 2, b1, &full[stage], kb * GEMM_BK, r1);
+                    if (++stage == G_STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // Let copies already issued land before the CTA can exit.
+                for (int i = 0; i < G_STAGES; ++i) mbar_wait(&full[i], 0, nullptr, 0);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(GEMM_BM, GEMM_BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+                const int acc = it & 1;
+                const uint32_t acc_phase = (it >> 1) & 1;
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, err, DERR_GEMM_MMA_WAIT)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * GEMM_BN;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, err, DERR_GEMM_MMA_WAIT)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + stage * G_STAGE_BYTES);
+                    const uint32_t sb = sa + G_A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
+                        tc_mma_f16(d_tmem, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32), idesc,
+                                   (kb | kk) != 0);
+                    }
+                    tc_commit(&empty[stage]);
+                    if (++stage == G_STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                tc_commit(&tfull[acc]);
+            }
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5) ----------------
+        const int quarter = warp & 3;  // TMEM lanes this warp may access
+        const int row_in_tile = quarter * 32 + lane;
+        const Epi& e = p.epi;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+            const int mb = tile % num_m, nb = tile / num_m;
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            if (!mbar_wait(&tfull[acc], acc_phase, err, DERR_GEMM_EPI_WAIT)) break;
+            tc_fence_after();
+            const int m = mb * GEMM_BM + row_in_tile;
+            const bool valid = m < p.M;
+            const float rinv = valid ? row_rinv(e.norm, m) : 0.f;
+            const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * GEMM_BN;
+            if (EPI == EPI_SWIGLU) {
+                const int n0 = nb * (GEMM_BN / 2);
+#pragma unroll 1
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t ra[32], rc[32];
+                    tc_ld_32x32b_x32(tbase + ch * 32, ra);
+                    tc_ld_32x32b_x32(tbase + GEMM_BN / 2 + ch * 32, rc);
+                    tc_wait_ld();
+                    if (valid) {
+                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(e.g_out) + (size_t)m * e.F + n0 + ch * 32;
+#pragma unroll
+                        for (int j = 0; j < 32; j += 8) {
+                            float v[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                v[i] = swiglu(__uint_as_float(ra[j + i]) * rinv, __uint_as_float(rc[j + i]) * rinv);
+                            store8<__nv_bfloat16>(dst + j, v);
+                        }
+                    }
+                }
+            } else {
+                float ss = 0.f;
+#pragma unroll 1
+                for (int ch = 0; ch < GEMM_BN / 32; ++ch) {
+                    uint32_t r[32];
+                    tc_ld_32x32b_x32(tbase + ch * 32, r);
+                    tc_wait_ld();
+                    if (!valid) continue;
+                    const int c0 = nb * GEMM_BN + ch * 32;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8) {
+                        float v[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[j + i]) * rinv;
+                        if (EPI == EPI_STORE_F32) {
+                            store8<float>(e.y + (size_t)m * e.ldy + c0 + j, v);
+                        } else if (EPI == EPI_QKV_ROPE) {
+                            epi_qkv8<__nv_bfloat16>(e, m, c0 + j, v);
+                        } else if (EPI == EPI_RESID) {
+                            float* hp = e.h + (size_t)m * e.D + c0 + j;
+                            const float4 h0 = reinterpret_cast<const float4*>(hp)[0];
+                            const float4 h1 = reinterpret_cast<const float4*>(hp)[1];
+                            float hn[8] = {h0.x + v[0], h0.y + v[1], h0.z + v[2], h0.w + v[3],
+                                           h1.x + v[4], h1.y + v[5], h1.z + v[6], h1.w + v[7]};
+                            store8<float>(hp, hn);
+                            const uint4 wv = *reinterpret_cast<const uint4*>(
+                                reinterpret_cast<const __nv_bfloat16*>(e.wnext) + c0 + j);
+                            float hw[8];
+                            hw[0] = hn[0] * bf16lo(wv.x);
+                            hw[1] = hn[1] * bf16hi(wv.x);
+                            hw[2] = hn[2] * bf16lo(wv.y);
+                            hw[3] = hn[3] * bf16hi(wv.y);
+                            hw[4] = hn[4] * bf16lo(wv.z);
+                            hw[5] = hn[5] * bf16hi(wv.z);
+                            hw[6] = hn[6] * bf16lo(wv.w);
+                            hw[7] = hn[7] * bf16hi(wv.w);
+                            store8<__nv_bfloat16>(reinterpret_cast<__nv_bfloat16*>(e.hw_out) + (size_t)m * e.D + c0 + j,
+                                                  hw);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) ss += hn[i] * hn[i];
+                        }
+                    }
+                }
+                if (EPI == EPI_RESID && valid) e.ss_out[(size_t)nb * e.ss_out_ld + m] = ss;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tc_dealloc(tmem_base, G_TMEM_COLS);
+    }
+}
+
+cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t s, bool pdl) {
+    if (a.M < 1 || a.K % GEMM_BK != 0) return cudaErrorInvalidValue;
+    const int kind = a.epi.kind;
+    if (kind == EPI_SWIGLU ? (a.N % (GEMM_BN / 2) != 0) : (a.N % GEMM_BN != 0)) return cudaErrorInvalidValue;
+    if (kind == EPI_LOGITS) return cudaErrorInvalidValue;
+    GemmKernelParams p;
+    for (int i = 0; i < 3; ++i) p.seg_cols[i] = a.seg_cols[i];
+    p.M = a.M;
+    p.N = a.N;
+    p.K = a.K;
+    p.epi = a.epi;
+    const int num_m = (a.M + GEMM_BM - 1) / GEMM_BM;
+    const int num_n = kind == EPI_SWIGLU ? a.N / (GEMM_BN / 2) : a.N / GEMM_BN;
+    const int total = num_m * num_n;
+    const dim3 grid(total < a.num_sms ? total : a.num_sms);
+    const CUtensorMap& b0 = *a.tmB[0];
+    const CUtensorMap& b1 = a.tmB[1] ? *a.tmB[1] : *a.tmB[0];
+    const CUtensorMap& b2 = a.tmB[2] ? *a.tmB[2] : *a.tmB[0];
+    auto go = [&](auto kern) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        return launch_k(kern, grid, dim3(G_THREADS), G_SMEM_BYTES, s, pdl, *a.tmA, b0, b1, b2, p);
+    };
+    switch (kind) {
+        case EPI_STORE_F32: return go(gemm_tc_kernel<EPI_STORE_F32>);
+        case EPI_QKV_ROPE: return go(gemm_tc_kernel<EPI_QKV_ROPE>);
+        case EPI_SWIGLU: return go(gemm_tc_kernel<EPI_SWIGLU>);
+        case EPI_RESID: return go(gemm_tc_kernel<EPI_RESID>);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace lfw

@@ -1,0 +1,177 @@
+// Parameter blocks and host launchers of the decoder's kernels.
+//
+// Data layout in device memory (one model):
+//   h      fp32 [tokens][dim]            residual stream
+//   hw     act  [tokens][dim]            h * (next RMSNorm weight), the projection input;
+//                                        its per-row RMS scale is applied in the consumer's epilogue
+//   ss     fp32 [parts][ss_ld]           partial sums of h^2 per row, written by the producer of h
+//   q      act  [tokens][n_heads*head_dim]      post-RoPE queries
+//   o      act  [tokens][n_heads*head_dim]      attention output (heads concatenated)
+//   g      act  [tokens][ffn_hidden]     silu(w1 x) * (w3 x)
+//   K, V   act  [layer][batch][kv_head][position][head_dim]
+// "act" is bf16 for bf16 models and fp32 for fp32 models. A token row m belongs
+// to sequence b = m / T at position pos0[b] + (m % T).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <utility>
+
+namespace lfw {
+
+enum EpiKind : int {
+    EPI_STORE_F32 = 0,  // y[m][n] = acc
+    EPI_QKV_ROPE = 1,   // rotate q/k pairs, write q and append k, v to the cache
+    EPI_SWIGLU = 2,     // g[m][n] = silu(acc_w1) * acc_w3
+    EPI_RESID = 3,      // h[m][n] += acc; hw = h * wnext; partial sum of h^2
+    EPI_LOGITS = 4,     // logits (optional) + greedy argmax, last-CTA reduction
+};
+
+// The RMSNorm scale of a projection input that was stored as h * w:
+// rinv[m] = 1 / sqrt(sum_p ss[p * ld + row0 + m * row_step] / dim + eps).
+struct NormIn {
+    const float* ss = nullptr;  // nullptr: input is not normed (no scaling)
+    int nparts = 0, ld = 0, row0 = 0, row_step = 1;
+    float inv_dim = 0.f, eps = 0.f;
+};
+
+struct Epi {
+    int kind = EPI_STORE_F32;
+    int M = 0;  // output rows (tokens)
+    int T = 1;  // tokens per sequence
+    NormIn norm;
+    // EPI_STORE_F32
+    float* y = nullptr;
+    int ldy = 0;
+    // EPI_QKV_ROPE
+    const int32_t* pos0 = nullptr;
+    const float* rope_cos = nullptr;  // [max_seq][head_dim/2]
+    const float* rope_sin = nullptr;
+    int H = 0, Hk = 0, d = 0, S_max = 0;
+    void* q_out = nullptr;
+    void* k_cache = nullptr;  // this layer: [batch][Hk][S_max][d]
+    void* v_cache = nullptr;
+    // EPI_SWIGLU
+    void* g_out = nullptr;
+    int F = 0;
+    // EPI_RESID
+    float* h = nullptr;
+    int D = 0;
+    void* hw_out = nullptr;
+    const void* wnext = nullptr;
+    float* ss_out = nullptr;
+    int ss_out_ld = 0;
+    // EPI_LOGITS
+    float* logits = nullptr;
+    int ld_logits = 0;
+    float* am_val = nullptr;  // [tiles][M]
+    int* am_idx = nullptr;
+    unsigned* am_counter = nullptr;  // zero between launches; the last CTA resets it
+    int32_t* next_tok = nullptr;
+    int32_t* seq_len = nullptr;  // when set: seq_len[m] += advance, by the last CTA
+    int advance = 0;
+    uint32_t* err = nullptr;
+};
+
+// ---- decode projection: y = x W^T for M <= 16 token rows ---------------
+template <typename T>
+struct GemvArgs {
+    const T* W[3] = {nullptr, nullptr, nullptr};  // QKV: wq, wk, wv; SWIGLU: w1, w3; else W[0]
+    int seg_rows[3] = {0, 0, 0};                  // rows of each segment
+    int N = 0;                                    // logical output rows (SWIGLU: ffn_hidden)
+    int K = 0;
+    const T* x = nullptr;  // [M][ldx]
+    int ldx = 0;
+    int M = 0;   // rows in this launch (<= 16)
+    int m0 = 0;  // token index of row 0 (the epilogue sees token m0 + m)
+    Epi epi;
+};
+// Number of 16-row tiles (parts of the RESID partial sums, tiles of LOGITS partials).
+int gemv_num_tiles(int kind, int N);
+cudaError_t launch_gemv_bf16(const GemvArgs<__nv_bfloat16>& a, cudaStream_t s, bool pdl);
+cudaError_t launch_gemv_f32(const GemvArgs<float>& a, cudaStream_t s, bool pdl);
+
+// ---- prefill projection on tcgen05 ------------------------------------
+struct GemmArgs {
+    const CUtensorMap* tmA = nullptr;                          // activations [rows][K] bf16
+    const CUtensorMap* tmB[3] = {nullptr, nullptr, nullptr};   // weight segments [rows][K] bf16
+    int seg_cols[3] = {0, 0, 0};  // output columns of each segment (SWIGLU: seg 0 = ffn_hidden)
+    int M = 0, N = 0, K = 0;      // N: total output columns (SWIGLU: ffn_hidden)
+    int num_sms = 148;
+    Epi epi;
+};
+constexpr int GEMM_BM = 128, GEMM_BN = 256, GEMM_BK = 64;
+cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t s, bool pdl);
+
+// ---- attention --------------------------------------------------------
+struct AttnPrefillArgs {
+    const CUtensorMap* tmK = nullptr;  // 2-D view of the K cache: [rows][head_dim] bf16
+    const CUtensorMap* tmV = nullptr;
+    long long row_base = 0;            // cache row of (batch 0, kv head 0, position 0) of this layer
+    int S_max = 0;
+    const __nv_bfloat16* q = nullptr;  // [B*T][H*d]
+    __nv_bfloat16* out = nullptr;      // [B*T][H*d]
+    const int32_t* pos0 = nullptr;
+    int B = 0, T = 0, H = 0, Hk = 0;
+    float scale_log2 = 0.f;            // log2(e) / sqrt(d)
+    uint32_t* err = nullptr;
+};
+cudaError_t launch_attn_prefill(const AttnPrefillArgs& a, cudaStream_t s, bool pdl);
+
+struct AttnDecodeArgs {
+    const void* q = nullptr;   // [B*T][H*d]
+    const void* kc = nullptr;  // this layer: [batch][Hk][S_max][d]
+    const void* vc = nullptr;
+    void* out = nullptr;       // [B*T][H*d]
+    const int32_t* pos0 = nullptr;
+    int B = 0, T = 0, H = 0, Hk = 0, d = 0, S_max = 0;
+    int n_splits = 1, tq = 1, n_qchunks = 1;
+    float* ws_part = nullptr;       // split partials (m, l, o[d])
+    unsigned* ws_count = nullptr;   // [B*Hk*n_qchunks], zero between launches
+    float scale_log2 = 0.f;
+};
+struct AttnDecodePlan {
+    int n_splits, tq, n_qchunks;
+    size_t part_floats, counters;
+};
+AttnDecodePlan attn_decode_plan(int B, int T, int H, int Hk, int d, int max_keys, int num_sms);
+cudaError_t launch_attn_decode(const AttnDecodeArgs& a, bool bf16, cudaStream_t s, bool pdl);
+
+// ---- small kernels ----------------------------------------------------
+struct EmbedArgs {
+    const int32_t* tok = nullptr;  // token ids [M] (when h_in is null)
+    const void* E = nullptr;       // [vocab][D] model dtype
+    const float* h_in = nullptr;   // or given hidden states [M][D]
+    float* h = nullptr;
+    void* hw = nullptr;
+    const void* wnorm = nullptr;   // first layer's attention_norm
+    float* ss = nullptr;           // [1][M]
+    int M = 0, D = 0, vocab = 0;
+};
+cudaError_t launch_embed(const EmbedArgs& a, bool bf16, cudaStream_t s, bool pdl);
+// h_out = h; seq_len[b] += advance for b < B.
+cudaError_t launch_finish_hidden(const float* h, float* h_out, long long n, int32_t* seq_len, int B,
+                                 int advance, cudaStream_t s, bool pdl);
+cudaError_t launch_rope_tables(float* cosv, float* sinv, int n_pos, int half, double theta, int head_dim,
+                               cudaStream_t s);
+
+// Launch helper: programmatic stream serialization when pdl is set.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                     Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+}  // namespace lfw

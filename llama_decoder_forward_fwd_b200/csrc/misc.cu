@@ -1,0 +1,94 @@
+// Small kernels at the ends of a pass: the embedding lookup that starts the
+// residual stream, the hidden-state output of the layer-stack-only path, and the
+// RoPE cos/sin tables built once at model creation.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace lfw {
+
+constexpr int EMB_THREADS = 256;
+
+// h[m] = E[tok[m]] ("Building llama3 from scratch": the embedding layer maps each
+// token id to its row of tok_embeddings) or the given hidden state, plus the first
+// layer's RMSNorm inputs: hw[m] = h[m] * w and ss[m] = sum h[m]^2.
+template <typename WT>
+__global__ void __launch_bounds__(EMB_THREADS) embed_kernel(const EmbedArgs a) {
+    __shared__ float red[EMB_THREADS / 32];
+    const int m = blockIdx.x;
+    pdl_trigger();
+    pdl_wait();
+    const WT* wn = reinterpret_cast<const WT*>(a.wnorm);
+    WT* hw = reinterpret_cast<WT*>(a.hw) + (long long)m * a.D;
+    float* h = a.h + (long long)m * a.D;
+    const WT* src = nullptr;
+    const float* hsrc = nullptr;
+    if (a.h_in) {
+        hsrc = a.h_in + (long long)m * a.D;
+    } else {
+        int tok = a.tok[m];
+        tok = tok < 0 ? 0 : (tok >= a.vocab ? a.vocab - 1 : tok);
+        src = reinterpret_cast<const WT*>(a.E) + (long long)tok * a.D;
+    }
+    float ss = 0.f;
+    for (int i = threadIdx.x; i < a.D; i += EMB_THREADS) {
+        const float v = hsrc ? hsrc[i] : to_f<WT>(src[i]);
+        h[i] = v;
+        hw[i] = from_f<WT>(v * to_f<WT>(wn[i]));
+        ss += v * v;
+    }
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float t = 0.f;
+        for (int w = 0; w < EMB_THREADS / 32; ++w) t += red[w];
+        a.ss[m] = t;
+    }
+}
+
+cudaError_t launch_embed(const EmbedArgs& a, bool bf16, cudaStream_t s, bool pdl) {
+    if (bf16) return launch_k(embed_kernel<__nv_bfloat16>, dim3(a.M), EMB_THREADS, 0, s, pdl, a);
+    return launch_k(embed_kernel<float>, dim3(a.M), EMB_THREADS, 0, s, pdl, a);
+}
+
+__global__ void finish_hidden_kernel(const float* h, float* h_out, long long n, int32_t* seq_len, int B,
+                                     int advance) {
+    pdl_trigger();
+    pdl_wait();
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+        h_out[i] = h[i];
+    if (blockIdx.x == 0 && threadIdx.x < B) seq_len[threadIdx.x] += advance;
+}
+
+cudaError_t launch_finish_hidden(const float* h, float* h_out, long long n, int32_t* seq_len, int B, int advance,
+                                 cudaStream_t s, bool pdl) {
+    long long blocks = (n + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    if (blocks < 1) blocks = 1;
+    return launch_k(finish_hidden_kernel, dim3((unsigned)blocks), dim3(256), 0, s, pdl, h, h_out, n, seq_len, B,
+                    advance);
+}
+
+// cos/sin of p * theta^(-2i/head_dim) for p < n_pos, i < head_dim/2 (llama3.np
+// page, "RoPE #1": positions times frequencies, then cos and sin), evaluated in
+// double precision and stored as fp32.
+__global__ void rope_table_kernel(float* cosv, float* sinv, int n_pos, int half, double theta, int head_dim) {
+    const long long n = (long long)n_pos * half;
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const int p = (int)(idx / half), i = (int)(idx % half);
+        const double freq = pow(theta, -2.0 * i / head_dim);
+        double sn, cs;
+        sincos((double)p * freq, &sn, &cs);
+        cosv[idx] = (float)cs;
+        sinv[idx] = (float)sn;
+    }
+}
+
+cudaError_t launch_rope_tables(float* cosv, float* sinv, int n_pos, int half, double theta, int head_dim,
+                               cudaStream_t s) {
+    rope_table_kernel<<<256, 256, 0, s>>>(cosv, sinv, n_pos, half, theta, head_dim);
+    return cudaGetLastError();
+}
+
+}  // namespace lfw

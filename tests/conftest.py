@@ -24,4 +24,6 @@ def gpu_available() -> bool:
 def lib():
     """The built CUDA library's Python binding (building it first when missing)."""
     import llama_decoder_forward_fwd_b200 as L
+    from llama_decoder_forward_fwd_b200 import build
+    build.build()
     return L.load()

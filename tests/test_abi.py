@@ -1,0 +1,88 @@
+"""The C-ABI library builds, loads, and exports every symbol include/*.h declares.
+
+CPU only: no call here reaches a CUDA kernel. The negative calls below are
+rejected by host-side argument checks before any CUDA API is used.
+"""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import llama_decoder_forward_fwd_b200 as L
+from llama_decoder_forward_fwd_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"\b(llm_\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.load()
+
+
+def test_header_declares_the_boundary_calls():
+    names = declared_functions()
+    for required in ("llm_model_init", "llm_prefill", "llm_decode_step", "llm_kv_cache_reset", "llm_model_free"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_covers_every_declared_symbol():
+    assert sorted(L.exported_symbols()) == declared_functions()
+
+
+def test_config_struct_layout_matches_header():
+    # 10 ints, 2 floats, 4 ints
+    assert ctypes.sizeof(L.llm_config) == 16 * 4
+    assert ctypes.sizeof(L.llm_weights) == 12 * ctypes.sizeof(ctypes.c_void_p)
+
+
+def test_null_arguments_are_rejected_on_the_host(lib):
+    h = ctypes.c_void_p()
+    assert lib.llm_model_init(None, None, None, ctypes.byref(h)) == L.LLM_ERR_NULL_PTR
+    assert h.value is None
+    assert lib.llm_model_init(None, None, None, None) == L.LLM_ERR_NULL_PTR
+    assert b"NULL" in lib.llm_last_error()
+    assert lib.llm_prefill(None, None, 1, 1, None, None) == L.LLM_ERR_NULL_PTR
+    assert lib.llm_decode_step(None, 1, None, None, None) == L.LLM_ERR_NULL_PTR
+    assert lib.llm_kv_cache_reset(None) == L.LLM_ERR_NULL_PTR
+    assert lib.llm_synchronize(None) == L.LLM_ERR_NULL_PTR
+    assert lib.llm_op_gemm_bf16(None, None, None, 1, 256, 64, None) == L.LLM_ERR_NULL_PTR
+    lib.llm_model_free(None)
+
+
+def test_inconsistent_configs_are_rejected_on_the_host(lib):
+    import seeded_inputs as S
+    shape = S.WORKLOADS["llama3-8b-bf16-b1-p2048-g256"].shape
+    w = L.llm_weights()
+    h = ctypes.c_void_p()
+    bad = [dict(n_kv_heads=5), dict(head_dim=64), dict(dtype=7), dict(max_batch=0), dict(max_batch=17)]
+    for kw in bad:
+        cfg = L.make_config(shape, max_batch=1)
+        for k, v in kw.items():
+            setattr(cfg, k, v)
+        assert lib.llm_model_init(ctypes.byref(cfg), ctypes.byref(w), None, ctypes.byref(h)) == L.LLM_ERR_BAD_CONFIG, kw
+
+
+def test_op_shape_checks_are_host_side(lib):
+    p = ctypes.c_void_p(16)  # never dereferenced: the shape check fails first
+    assert lib.llm_op_gemm_bf16(p, p, p, 4, 100, 64, None) == L.LLM_ERR_BAD_ARG     # N % 256
+    assert lib.llm_op_gemm_bf16(p, p, p, 4, 256, 60, None) == L.LLM_ERR_BAD_ARG     # K % 64
+    assert lib.llm_op_gemv_bf16(p, p, p, 17, 16, 64, None) == L.LLM_ERR_BAD_ARG     # M > 16
+    assert lib.llm_op_attention_decode_workspace(1, 1, 32, 8, 128) > 0
+    assert lib.llm_op_attention_decode_workspace(1, 1, 30, 8, 128) == 0             # H % Hk

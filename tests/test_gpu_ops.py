@@ -1,0 +1,110 @@
+"""Single-kernel parity against fp64 definitions, through the C ABI (GPU).
+
+Expected values are the plain definitions in float64 on the same bf16/fp32
+inputs: the projection y = x W^T, and causal GQA attention from the oracle.
+Tolerances follow from the arithmetic (fp32 accumulation; bf16 rounding of the
+softmax weights and of the output), stated per test.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _rand(shape, dtype, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g) * scale).to(dtype)
+
+
+def _proj_check(x, W, y_gpu, rel=2e-5):
+    """|y - x W^T| <= rel * (|x| |W|^T) + 1e-6: fp32 accumulation of K bf16 products."""
+    x64, w64 = O.f64(x), O.f64(W)
+    ref = x64 @ w64.T
+    bound = rel * (np.abs(x64) @ np.abs(w64).T) + 1e-6
+    err = np.abs(O.f64(y_gpu) - ref)
+    assert np.all(err <= bound), f"max err {err.max():.3e}, worst ratio {(err / bound).max():.2f}"
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 64), (100, 512, 128), (128, 256, 4096), (300, 768, 1024),
+                                   (2048, 1024, 4096), (129, 256, 14336)])
+def test_gemm_tcgen05_matches_definition(lib, M, N, K):
+    import llama_decoder_forward_fwd_b200 as L
+    A = _rand((M, K), torch.bfloat16, 1).to(DEV)
+    B = _rand((N, K), torch.bfloat16, 2, 0.02).to(DEV)
+    C = torch.full((M, N), float("nan"), device=DEV)
+    L.llm_op_gemm_bf16(A, B, C)
+    torch.cuda.synchronize()
+    _proj_check(A.cpu(), B.cpu(), C.cpu())
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 16, 64), (1, 4096, 4096), (3, 100, 200), (8, 1024, 14336),
+                                   (9, 64, 1024), (16, 4096, 4096), (1, 32000, 4096)])
+def test_gemv_matches_definition(lib, M, N, K):
+    import llama_decoder_forward_fwd_b200 as L
+    x = _rand((M, K), torch.bfloat16, 3).to(DEV)
+    W = _rand((N, K), torch.bfloat16, 4, 0.02).to(DEV)
+    y = torch.full((M, N), float("nan"), device=DEV)
+    L.llm_op_gemv_bf16(x, W, y)
+    torch.cuda.synchronize()
+    _proj_check(x.cpu(), W.cpu(), y.cpu())
+
+
+def _attn_case(B, T, H, Hk, d, S_max, pos0, dtype, seed):
+    q = _rand((B, T, H, d), dtype, seed)
+    kc = _rand((B, Hk, S_max, d), dtype, seed + 1)
+    vc = _rand((B, Hk, S_max, d), dtype, seed + 2)
+    ref = np.empty((B, T, H * d))
+    for b in range(B):
+        n = pos0[b] + T
+        qp = pos0[b] + np.arange(T)
+        k = O.f64(kc[b, :, :n, :]).transpose(1, 0, 2)
+        v = O.f64(vc[b, :, :n, :]).transpose(1, 0, 2)
+        ref[b] = O.attention(O.f64(q[b]), k, v, qp, np.arange(n))
+    return q, kc, vc, ref
+
+
+ATTN_CASES = [
+    # B, T, H, Hk, pos0
+    (1, 1, 32, 8, [0]),
+    (2, 7, 8, 2, [0, 5]),
+    (2, 130, 8, 2, [0, 64]),
+    (1, 300, 32, 8, [0]),
+    (2, 64, 4, 4, [3, 0]),
+]
+
+
+@pytest.mark.parametrize("B,T,H,Hk,pos0", ATTN_CASES)
+def test_flash_attention_prefill_matches_oracle(lib, B, T, H, Hk, pos0):
+    import llama_decoder_forward_fwd_b200 as L
+    d, S = 128, 512
+    q, kc, vc, ref = _attn_case(B, T, H, Hk, d, S, pos0, torch.bfloat16, 11)
+    out = torch.full((B, T, H * d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    p = torch.tensor(pos0, dtype=torch.int32, device=DEV)
+    L.llm_op_attention_prefill(q.to(DEV), kc.to(DEV), vc.to(DEV), p, out)
+    torch.cuda.synchronize()
+    # softmax weights and the output are rounded to bf16: |err| <= 3 * 2^-9 * max|v|.
+    err = np.abs(O.f64(out.cpu()) - ref)
+    assert err.max() <= 8e-3 * float(vc.abs().max()), err.max()
+
+
+@pytest.mark.parametrize("dtype,d,tol", [(torch.bfloat16, 128, 6e-3), (torch.float32, 48, 2e-5),
+                                         (torch.float32, 128, 2e-5)])
+@pytest.mark.parametrize("B,T,H,Hk,pos0", [(1, 1, 32, 8, [0]), (3, 1, 32, 8, [0, 37, 700]),
+                                           (2, 4, 8, 2, [9, 0]), (1, 8, 6, 6, [0]), (2, 3, 12, 3, [100, 1])])
+def test_split_kv_attention_matches_oracle(lib, dtype, d, tol, B, T, H, Hk, pos0):
+    import llama_decoder_forward_fwd_b200 as L
+    S = 1024
+    q, kc, vc, ref = _attn_case(B, T, H, Hk, d, S, pos0, dtype, 21)
+    out = torch.full((B, T, H * d), float("nan"), dtype=dtype, device=DEV)
+    p = torch.tensor(pos0, dtype=torch.int32, device=DEV)
+    ws = torch.empty(L.llm_op_attention_decode_workspace(B, T, H, Hk, d), dtype=torch.uint8, device=DEV)
+    for _ in range(2):  # the second call reuses the workspace the first left behind
+        L.llm_op_attention_decode(q.to(DEV), kc.to(DEV), vc.to(DEV), p, out, ws)
+    torch.cuda.synchronize()
+    err = np.abs(O.f64(out.cpu()) - ref)
+    assert err.max() <= tol * float(vc.abs().max()), err.max()
