@@ -619,7 +619,7 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
     if (c.flags & LLM_FLAG_DEBUG_TAPS) MALLOC_OR_BAIL(m->taps, (size_t)c.n_layers * Mx * D * 4);
 
     if (cudaMemsetAsync(m->am_counter, 0, 64, m->stream) != cudaSuccess ||
-        cudaMemsetAsync(m->attn_cnt, 0, m->attn_cnt_n * 4 + 4, m->stream) != cudaSuccess ||
+        cudaMemsetAsync(m->attn_cnt, 0, m->attn_cnt_n * 4, m->stream) != cudaSuccess ||
         cudaMemsetAsync(m->seq_len, 0, (size_t)c.max_batch * 4, m->stream) != cudaSuccess ||
         cudaMemsetAsync(m->d_err, 0, 64, m->stream) != cudaSuccess ||
         cudaMemsetAsync(m->ss, 0, (size_t)parts * Mx * 4, m->stream) != cudaSuccess)
