@@ -319,7 +319,7 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- per-kernel CUDA-event timing of one step (roofline of the dominant kernel) ----
     tm = L.Model(shape, model.glob, model.layers, max_batch=B, max_tokens=B * T,
-                 flags=L.LLM_FLAG_KERNEL_TIMING, stream=stream, device=dev)
+                 flags=L.LLM_FLAG_KERNEL_TIMING | L.LLM_FLAG_CUDA_GRAPH, stream=stream, device=dev)
     gen2 = torch.zeros_like(gen)
     L.llm_prefill(tm.h, prompt, gen2[0])
     kt_pre = L.llm_kernel_times(tm.h, reset=True)

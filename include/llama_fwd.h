@@ -60,7 +60,11 @@ extern "C" {
 #define LLM_FLAG_CUDA_GRAPH  1  /* replay decode steps from captured CUDA graphs */
 #define LLM_FLAG_DEBUG_TAPS  2  /* keep each layer's output hidden state (see llm_debug_tap) */
 #define LLM_FLAG_KERNEL_TIMING 4 /* time every launch with CUDA events (see llm_kernel_times);
-                                    ignored for graph-replayed decode steps */
+                                    with LLM_FLAG_CUDA_GRAPH the events are nodes of the decode
+                                    graph and each decode step synchronises to read them */
+#define LLM_FLAG_PDL           8 /* let each kernel launch while the previous one drains
+                                    (programmatic dependent launch); off by default because it
+                                    unbalances the persistent one-CTA-per-SM projections */
 
 /* ---- kernel kinds reported by llm_kernel_times ------------------------- */
 #define LLM_K_EMBED    0   /* embedding lookup / hidden-state load */
@@ -142,7 +146,8 @@ int llm_prefill(llm_model* m, const int32_t* tokens, int B, int T, int32_t* next
 /*
  * Prefill of the layer stack on given hidden states, with no embedding, final
  * norm or lm_head. h_in: device fp32 [B, T, dim]; h_out: device fp32 [B, T, dim],
- * the last layer's output. Positions and cache growth as in llm_prefill.
+ * the last layer's output; both 16-byte aligned (else LLM_ERR_BAD_ARG).
+ * Positions and cache growth as in llm_prefill.
  */
 int llm_prefill_hidden(llm_model* m, const float* h_in, int B, int T, float* h_out);
 
@@ -188,7 +193,9 @@ int llm_debug_tap(llm_model* m, int layer, float* dst, size_t dst_elems);
  * kinds 0..n-1 (see LLM_K_*) into the host arrays total_ms[n] and launches[n];
  * reset != 0 clears the record afterwards. Kernels are timed with a CUDA event
  * pair each on the model's stream, so kernels that would otherwise overlap
- * their neighbours' tails run back to back while timing is on.
+ * their neighbours' tails run back to back while timing is on. Directly
+ * launched kernels include any host launch gap in their time; decode steps
+ * replayed from a graph (LLM_FLAG_CUDA_GRAPH) do not.
  */
 int llm_kernel_times(llm_model* m, int n, double* total_ms, int64_t* launches, int reset);
 
@@ -216,11 +223,17 @@ const char* llm_last_error(void);
 int llm_op_gemm_bf16(const void* A, const void* B, float* C, int M, int N, int K, void* stream);
 
 /*
- * y = x W^T for a few rows (the decode projection kernel). x: device bf16
- * [M, K] with M <= 16; W: device bf16 [N, K]; y: device fp32 [M, N].
- * Needs K % 8 == 0.
+ * y = x W^T for a few rows (the decode projection kernel, streaming W once).
+ * x: device bf16 [M, K] with M <= 16; W: device bf16 [N, K]; y: device fp32
+ * [M, N]. Needs K % 8 == 0. workspace: device scratch of at least
+ * llm_op_gemv_workspace(N, K) bytes, 16-byte aligned, contents arbitrary (the
+ * call clears the part it needs); calls sharing one workspace must not overlap
+ * in time. Source: the per-token projection q_per_token = x @ wq_head^T of
+ * "Building llama3 from scratch", for the decode phase of llama3.np "Generasi".
  */
-int llm_op_gemv_bf16(const void* x, const void* W, float* y, int M, int N, int K, void* stream);
+size_t llm_op_gemv_workspace(int N, int K);
+int llm_op_gemv_bf16(const void* x, const void* W, float* y, int M, int N, int K, void* workspace,
+                     size_t workspace_bytes, void* stream);
 
 /*
  * Causal grouped-query attention over a KV cache for a block of new tokens

@@ -29,6 +29,7 @@ LLM_BF16 = 1
 LLM_FLAG_CUDA_GRAPH = 1
 LLM_FLAG_DEBUG_TAPS = 2
 LLM_FLAG_KERNEL_TIMING = 4
+LLM_FLAG_PDL = 8
 KERNEL_KINDS = ("embed", "qkv", "attn", "wo", "w13", "w2", "head", "out")
 
 
@@ -72,7 +73,8 @@ _SIGS = {
     "llm_model_free": (None, [_vp]),
     "llm_last_error": (ctypes.c_char_p, []),
     "llm_op_gemm_bf16": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
-    "llm_op_gemv_bf16": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
+    "llm_op_gemv_workspace": (_sz, [_i, _i]),
+    "llm_op_gemv_bf16": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp]),
     "llm_op_attention_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "llm_op_attention_decode_workspace": (_sz, [_i, _i, _i, _i, _i]),
     "llm_op_attention_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
@@ -190,10 +192,15 @@ def llm_op_gemm_bf16(A, B, C, stream=None):
     check(load().llm_op_gemm_bf16(_ptr(A), _ptr(B), _ptr(C), M, N, K, _stream_ptr(stream)))
 
 
-def llm_op_gemv_bf16(x, W, y, stream=None):
+def llm_op_gemv_workspace(N, K) -> int:
+    return load().llm_op_gemv_workspace(N, K)
+
+
+def llm_op_gemv_bf16(x, W, y, workspace, stream=None):
     M, K = x.shape
     N = W.shape[0]
-    check(load().llm_op_gemv_bf16(_ptr(x), _ptr(W), _ptr(y), M, N, K, _stream_ptr(stream)))
+    check(load().llm_op_gemv_bf16(_ptr(x), _ptr(W), _ptr(y), M, N, K, _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream_ptr(stream)))
 
 
 def _dt(t: torch.Tensor) -> int:

@@ -12,8 +12,8 @@
 //                  w2 projection + residual (writes hw = h * next norm weight, ss)
 //   head           last-position lm_head with RMSNorm scale + argmax (+ cache lengths)
 // Projections of more than 16 tokens run on the tcgen05 GEMM (bf16), otherwise on
-// the streaming decode GEMV. Every launch uses programmatic dependent launch so a
-// kernel's prologue (weight streaming) overlaps the previous kernel's tail.
+// the streaming decode GEMV. With LLM_FLAG_PDL, launches use programmatic
+// dependent launch so a kernel's prologue overlaps the previous kernel's tail.
 #include "../../include/llama_fwd.h"
 #include "kernels.cuh"
 
@@ -91,7 +91,11 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 struct LayerW {
     const void *attn_norm, *wq, *wk, *wv, *wo, *ffn_norm, *w1, *w3, *w2;
 };
-enum { TM_WQ, TM_WK, TM_WV, TM_WO, TM_W1, TM_W3, TM_W2, TM_PER_LAYER };
+enum { TM_WQ, TM_WK, TM_WV, TM_WO, TM_W1, TM_W3, TM_W2, TM_W1G, TM_W3G, TM_PER_LAYER };
+
+// RMSNorm partial sums written by a residual projection with N output rows.
+int bf16_gemv_ss_parts(int N) { return gemv_num_tiles(EPI_RESID, N) * 8; }  // one per 16 rows of a 128-row tile
+int f32_gemv_ss_parts(int N) { return (N + 15) / 16; }                     // one per CTA of 16 rows
 
 __device__ uint32_t g_op_err;  // device error word of the single-operation entry points
 
@@ -119,6 +123,7 @@ struct llm_model {
     float* am_val = nullptr;
     int* am_idx = nullptr;
     unsigned* am_counter = nullptr;
+    GemvScratch gws;
     float* attn_ws = nullptr;
     unsigned* attn_cnt = nullptr;
     size_t attn_ws_floats = 0, attn_cnt_n = 0;
@@ -129,20 +134,28 @@ struct llm_model {
     int taps_tokens = 0;
     std::vector<int> host_len;
     // tensor maps (bf16 models)
-    CUtensorMap tm_hw, tm_o, tm_g, tm_kc, tm_vc;
+    CUtensorMap tm_hw, tm_o, tm_g, tm_kc, tm_vc, tm_head;
     std::vector<CUtensorMap> tm_w;
     bool gemm_ok = false;
     // per-launch CUDA-event timing (LLM_FLAG_KERNEL_TIMING)
     bool timing = false;
     bool capturing = false;
+    bool pdl = false;  // programmatic dependent launch between consecutive kernels
     struct TimeRec {
         int kind;
         cudaEvent_t a, b;
     };
-    std::vector<TimeRec> trecs;
+    std::vector<TimeRec> trecs;      // direct launches since the last report
+    std::vector<TimeRec> cap_recs;   // event nodes of the graph being captured
+    double kt_ms[LLM_K_COUNT] = {};  // accumulated from graph replays
+    int64_t kt_n[LLM_K_COUNT] = {};
     std::vector<cudaEvent_t> ev_pool;
     // decode graphs keyed by (B, n_splits, logits requested)
-    std::map<std::tuple<int, int, int>, cudaGraphExec_t> graphs;
+    struct Graph {
+        cudaGraphExec_t exec;
+        std::vector<TimeRec> recs;  // timing event pairs inside the graph
+    };
+    std::map<std::tuple<int, int, int>, Graph> graphs;
     std::vector<void*> allocs;
 };
 
@@ -159,22 +172,30 @@ cudaEvent_t pool_event(llm_model* m) {
     return e;
 }
 
-// Brackets one kernel launch with an event pair when timing is on.
+// Brackets one kernel launch with an event pair when timing is on. Inside a
+// graph capture the events become event-record nodes of the graph, so each
+// replay timestamps the kernel on the device with no host gap in between.
 struct KTimer {
     llm_model* m;
     int kind;
     cudaEvent_t a = nullptr;
     KTimer(llm_model* mm, int k) : m(mm), kind(k) {
-        if (m->timing && !m->capturing && m->trecs.size() < 1000000) {
+        if (m->timing && m->trecs.size() < 1000000) {
             a = pool_event(m);
-            cudaEventRecord(a, m->stream);
+            if (m->capturing) cudaEventRecordWithFlags(a, m->stream, cudaEventRecordExternal);
+            else cudaEventRecord(a, m->stream);
         }
     }
     ~KTimer() {
         if (a) {
             cudaEvent_t b = pool_event(m);
-            cudaEventRecord(b, m->stream);
-            m->trecs.push_back({kind, a, b});
+            if (m->capturing) {
+                cudaEventRecordWithFlags(b, m->stream, cudaEventRecordExternal);
+                m->cap_recs.push_back({kind, a, b});
+            } else {
+                cudaEventRecord(b, m->stream);
+                m->trecs.push_back({kind, a, b});
+            }
         }
     }
 };
@@ -199,6 +220,8 @@ int validate_config(const llm_config* c) {
     if (c->has_embed_and_head && c->vocab <= 0) return fail(LLM_ERR_BAD_CONFIG, "vocab must be positive");
     if (c->n_heads / c->n_kv_heads > 16) return fail(LLM_ERR_BAD_CONFIG, "more than 16 query heads per KV head");
     if (c->max_batch > 16) return fail(LLM_ERR_BAD_CONFIG, "max_batch > 16");
+    if (c->dtype == LLM_BF16 && ((c->n_heads * c->head_dim) % 128 != 0 || (c->n_kv_heads * c->head_dim) % 128 != 0))
+        return fail(LLM_ERR_BAD_CONFIG, "bf16 models need n_heads*head_dim and n_kv_heads*head_dim multiples of 128");
     if (!(c->norm_eps >= 0.f) || !(c->rope_theta > 0.f)) return fail(LLM_ERR_BAD_CONFIG, "bad norm_eps or rope_theta");
     return LLM_OK;
 }
@@ -233,7 +256,7 @@ int project(llm_model* m, int l, int kind, int tkind, const void* x, const CUten
         ga.K = K;
         ga.num_sms = m->num_sms;
         ga.epi = epi;
-        CK(launch_gemm_tc(ga, m->stream, true));
+        CK(launch_gemm_tc(ga, m->stream, m->pdl));
         if (nparts_out) *nparts_out = c.dim / GEMM_BN;
         return LLM_OK;
     }
@@ -242,6 +265,12 @@ int project(llm_model* m, int l, int kind, int tkind, const void* x, const CUten
         if (m->bf16) {
             GemvArgs<__nv_bfloat16> ga;
             for (int i = 0; i < 3; ++i) ga.W[i] = reinterpret_cast<const __nv_bfloat16*>(W[i]);
+            for (int i = 0; i < 3; ++i) {
+                int t = tms[i];
+                if (kind == EPI_SWIGLU && t == TM_W1) t = TM_W1G;
+                if (kind == EPI_SWIGLU && t == TM_W3) t = TM_W3G;
+                ga.tmw[i] = t >= 0 ? &m->tm_w[(size_t)l * TM_PER_LAYER + t] : nullptr;
+            }
             for (int i = 0; i < 3; ++i) ga.seg_rows[i] = seg[i];
             ga.N = N;
             ga.K = K;
@@ -249,8 +278,10 @@ int project(llm_model* m, int l, int kind, int tkind, const void* x, const CUten
             ga.ldx = K;
             ga.M = rows;
             ga.m0 = r0;
+            ga.num_sms = m->num_sms;
+            ga.ws = m->gws;
             ga.epi = epi;
-            CK(launch_gemv_bf16(ga, m->stream, true));
+            CK(launch_gemv_bf16(ga, m->stream, m->pdl));
         } else {
             GemvArgs<float> ga;
             for (int i = 0; i < 3; ++i) ga.W[i] = reinterpret_cast<const float*>(W[i]);
@@ -262,10 +293,10 @@ int project(llm_model* m, int l, int kind, int tkind, const void* x, const CUten
             ga.M = rows;
             ga.m0 = r0;
             ga.epi = epi;
-            CK(launch_gemv_f32(ga, m->stream, true));
+            CK(launch_gemv_f32(ga, m->stream, m->pdl));
         }
     }
-    if (nparts_out) *nparts_out = gemv_num_tiles(kind, N);
+    if (nparts_out) *nparts_out = m->bf16 ? bf16_gemv_ss_parts(N) : f32_gemv_ss_parts(N);
     return LLM_OK;
 }
 
@@ -326,7 +357,7 @@ int run_layers(llm_model* m, int B, int T, int max_keys) {
             a.Hk = Hk;
             a.scale_log2 = scale_log2;
             a.err = m->d_err;
-            CK(launch_attn_prefill(a, m->stream, true));
+            CK(launch_attn_prefill(a, m->stream, m->pdl));
         } else {
             const AttnDecodePlan p = attn_decode_plan(B, T, H, Hk, d, max_keys, m->num_sms);
             if (p.part_floats > m->attn_ws_floats || p.counters > m->attn_cnt_n)
@@ -349,7 +380,8 @@ int run_layers(llm_model* m, int B, int T, int max_keys) {
             a.ws_part = m->attn_ws;
             a.ws_count = m->attn_cnt;
             a.scale_log2 = scale_log2;
-            CK(launch_attn_decode(a, m->bf16, m->stream, true));
+            a.err = m->d_err;
+            CK(launch_attn_decode(a, m->bf16, m->stream, m->pdl));
         }
         }
         // wo + residual; writes the ffn_norm input
@@ -429,8 +461,11 @@ int run_head(llm_model* m, int B, int T, int nparts, int32_t* next, float* logit
         ga.x = reinterpret_cast<const __nv_bfloat16*>(m->hw) + (size_t)(T - 1) * c.dim;
         ga.ldx = T * c.dim;
         ga.M = B;
+        ga.num_sms = m->num_sms;
+        ga.ws = m->gws;
+        ga.tmw[0] = &m->tm_head;
         ga.epi = e;
-        CK(launch_gemv_bf16(ga, m->stream, true));
+        CK(launch_gemv_bf16(ga, m->stream, m->pdl));
     } else {
         GemvArgs<float> ga;
         ga.W[0] = reinterpret_cast<const float*>(Wout);
@@ -440,7 +475,7 @@ int run_head(llm_model* m, int B, int T, int nparts, int32_t* next, float* logit
         ga.ldx = T * c.dim;
         ga.M = B;
         ga.epi = e;
-        CK(launch_gemv_f32(ga, m->stream, true));
+        CK(launch_gemv_f32(ga, m->stream, m->pdl));
     }
     return LLM_OK;
 }
@@ -448,7 +483,7 @@ int run_head(llm_model* m, int B, int T, int nparts, int32_t* next, float* logit
 int last_nparts(const llm_model* m, int M) {
     // Producer of the final hw/ss: the last layer's w2 projection.
     if (m->bf16 && M > 16 && m->gemm_ok) return m->cfg.dim / GEMM_BN;
-    return gemv_num_tiles(EPI_RESID, m->cfg.dim);
+    return m->bf16 ? bf16_gemv_ss_parts(m->cfg.dim) : f32_gemv_ss_parts(m->cfg.dim);
 }
 
 int check_batch(llm_model* m, int B, int T) {
@@ -481,7 +516,7 @@ int run_embed(llm_model* m, const int32_t* tok, const float* h_in, int M) {
     ea.D = m->cfg.dim;
     ea.vocab = m->cfg.vocab;
     KTimer timer(m, LLM_K_EMBED);
-    CK(launch_embed(ea, m->bf16, m->stream, true));
+    CK(launch_embed(ea, m->bf16, m->stream, m->pdl));
     return LLM_OK;
 }
 
@@ -503,7 +538,13 @@ const char* llm_last_error(void) { return g_last_error.c_str(); }
 void llm_model_free(llm_model* m) {
     if (!m) return;
     if (m->stream) cudaStreamSynchronize(m->stream);
-    for (auto& kv : m->graphs) cudaGraphExecDestroy(kv.second);
+    for (auto& kv : m->graphs) {
+        cudaGraphExecDestroy(kv.second.exec);
+        for (auto& r : kv.second.recs) {
+            cudaEventDestroy(r.a);
+            cudaEventDestroy(r.b);
+        }
+    }
     for (auto& r : m->trecs) {
         cudaEventDestroy(r.a);
         cudaEventDestroy(r.b);
@@ -542,6 +583,7 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
     m->M_max = m->cfg.max_tokens > c.max_batch ? m->cfg.max_tokens : c.max_batch;
     m->host_len.assign(c.max_batch, 0);
     m->timing = (c.flags & LLM_FLAG_KERNEL_TIMING) != 0;
+    m->pdl = (c.flags & LLM_FLAG_PDL) != 0;
     m->tok_emb = w->tok_emb;
     m->out = w->out;
     m->final_norm = w->final_norm;
@@ -575,14 +617,14 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
     MALLOC_OR_BAIL(m->o, Mx * H * d * es);
     MALLOC_OR_BAIL(m->g, Mx * F * es);
     m->ss_ld = (int)Mx;
-    const int parts = gemv_num_tiles(EPI_RESID, D) + 8;
+    const int parts = (bf16_gemv_ss_parts(D) > f32_gemv_ss_parts(D) ? bf16_gemv_ss_parts(D) : f32_gemv_ss_parts(D)) + 8;
     MALLOC_OR_BAIL(m->ss, (size_t)parts * Mx * 4);
     m->layer_elems = (long long)c.max_batch * Hk * c.max_seq_len * d;
     MALLOC_OR_BAIL(m->kc, (size_t)c.n_layers * m->layer_elems * es);
     MALLOC_OR_BAIL(m->vc, (size_t)c.n_layers * m->layer_elems * es);
     MALLOC_OR_BAIL(m->rope_cos, (size_t)c.max_seq_len * (d / 2) * 4);
     MALLOC_OR_BAIL(m->rope_sin, (size_t)c.max_seq_len * (d / 2) * 4);
-    const int vt = c.has_embed_and_head ? gemv_num_tiles(EPI_LOGITS, c.vocab) + 8 : 8;
+    const int vt = c.has_embed_and_head ? (c.vocab + 15) / 16 + 8 : 8;  // fp32 head: one argmax part per CTA
     MALLOC_OR_BAIL(m->am_val, (size_t)vt * c.max_batch * 4);
     MALLOC_OR_BAIL(m->am_idx, (size_t)vt * c.max_batch * 4);
     MALLOC_OR_BAIL(m->am_counter, 64);
@@ -611,6 +653,25 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
         MALLOC_OR_BAIL(m->attn_ws, pf * 4);
         MALLOC_OR_BAIL(m->attn_cnt, cn * 4);
     }
+    if (m->bf16) {
+        // Streaming GEMV scratch, sized for the largest projection of this model.
+        const int shapes[5][3] = {{EPI_QKV_ROPE, (H + 2 * Hk) * d, D}, {EPI_RESID, D, H * d}, {EPI_SWIGLU, F, D},
+                                  {EPI_RESID, D, F}, {EPI_LOGITS, c.has_embed_and_head ? c.vocab : 16, D}};
+        size_t pf = 0;
+        int tiles = 0;
+        for (auto& sh : shapes) {
+            const size_t f = gemv_scratch_floats(sh[0], sh[1], sh[2], m->num_sms);
+            pf = f > pf ? f : pf;
+            const int t = gemv_num_tiles(sh[0], sh[1]);
+            tiles = t > tiles ? t : tiles;
+        }
+        m->gws.part_floats = pf;
+        m->gws.tiles_cap = tiles;
+        MALLOC_OR_BAIL(m->gws.part, pf * 4);
+        MALLOC_OR_BAIL(m->gws.tile_cnt, (size_t)tiles * 4);
+        MALLOC_OR_BAIL(m->gws.am_best, 16 * 8);
+        MALLOC_OR_BAIL(m->gws.done_cnt, 16);
+    }
     MALLOC_OR_BAIL(m->d_tok, (size_t)c.max_batch * 4);
     MALLOC_OR_BAIL(m->d_next, (size_t)c.max_batch * 4);
     MALLOC_OR_BAIL(m->seq_len, (size_t)c.max_batch * 4);
@@ -622,33 +683,40 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
         cudaMemsetAsync(m->attn_cnt, 0, m->attn_cnt_n * 4, m->stream) != cudaSuccess ||
         cudaMemsetAsync(m->seq_len, 0, (size_t)c.max_batch * 4, m->stream) != cudaSuccess ||
         cudaMemsetAsync(m->d_err, 0, 64, m->stream) != cudaSuccess ||
-        cudaMemsetAsync(m->ss, 0, (size_t)parts * Mx * 4, m->stream) != cudaSuccess)
+        cudaMemsetAsync(m->ss, 0, (size_t)parts * Mx * 4, m->stream) != cudaSuccess ||
+        (m->bf16 && (cudaMemsetAsync(m->gws.tile_cnt, 0, (size_t)m->gws.tiles_cap * 4, m->stream) != cudaSuccess ||
+                     cudaMemsetAsync(m->gws.am_best, 0, 16 * 8, m->stream) != cudaSuccess ||
+                     cudaMemsetAsync(m->gws.done_cnt, 0, 16, m->stream) != cudaSuccess)))
         return bail(fail(LLM_ERR_CUDA, "cudaMemsetAsync failed"));
+    if (attn_decode_prepare() != cudaSuccess) return bail(fail(LLM_ERR_CUDA, "attention kernel attributes"));
     if (launch_rope_tables(m->rope_cos, m->rope_sin, c.max_seq_len, d / 2, (double)c.rope_theta, d, m->stream) !=
         cudaSuccess)
         return bail(fail(LLM_ERR_CUDA, "rope table kernel failed"));
 
-    // Tensor maps for the tcgen05 GEMM and the flash attention (bf16 only).
+    // Tensor maps (bf16 only): weights for the decode GEMV (128-row boxes, 64-row
+    // boxes of w1/w3 for the SwiGLU tiles) and the prefill GEMM, activations for
+    // the GEMM, the KV cache for the flash attention.
     if (m->bf16) {
-        bool ok = D % GEMM_BN == 0 && (H * d) % GEMM_BN == 0 && (Hk * d) % GEMM_BN == 0 && F % (GEMM_BN / 2) == 0 &&
-                  D % GEMM_BK == 0 && F % GEMM_BK == 0 && (H * d) % GEMM_BK == 0;
-        if (ok) {
-            ok = make_tmap(&m->tm_hw, m->hw, D, Mx, 64, 128) && make_tmap(&m->tm_o, m->o, H * d, Mx, 64, 128) &&
-                 make_tmap(&m->tm_g, m->g, F, Mx, 64, 128);
-            m->tm_w.resize((size_t)c.n_layers * TM_PER_LAYER);
-            for (int l = 0; l < c.n_layers && ok; ++l) {
-                CUtensorMap* t = &m->tm_w[(size_t)l * TM_PER_LAYER];
-                const LayerW& lw = m->L[l];
-                ok = make_tmap(&t[TM_WQ], lw.wq, D, (uint64_t)H * d, 64, 128) &&
-                     make_tmap(&t[TM_WK], lw.wk, D, (uint64_t)Hk * d, 64, 128) &&
-                     make_tmap(&t[TM_WV], lw.wv, D, (uint64_t)Hk * d, 64, 128) &&
-                     make_tmap(&t[TM_WO], lw.wo, (uint64_t)H * d, D, 64, 128) &&
-                     make_tmap(&t[TM_W1], lw.w1, D, F, 64, 128) && make_tmap(&t[TM_W3], lw.w3, D, F, 64, 128) &&
-                     make_tmap(&t[TM_W2], lw.w2, F, D, 64, 128);
-            }
-            if (!ok) return bail(fail(LLM_ERR_CUDA, "cuTensorMapEncodeTiled failed"));
+        bool ok = true;
+        m->tm_w.resize((size_t)c.n_layers * TM_PER_LAYER);
+        for (int l = 0; l < c.n_layers && ok; ++l) {
+            CUtensorMap* t = &m->tm_w[(size_t)l * TM_PER_LAYER];
+            const LayerW& lw = m->L[l];
+            ok = make_tmap(&t[TM_WQ], lw.wq, D, (uint64_t)H * d, 64, 128) &&
+                 make_tmap(&t[TM_WK], lw.wk, D, (uint64_t)Hk * d, 64, 128) &&
+                 make_tmap(&t[TM_WV], lw.wv, D, (uint64_t)Hk * d, 64, 128) &&
+                 make_tmap(&t[TM_WO], lw.wo, (uint64_t)H * d, D, 64, 128) &&
+                 make_tmap(&t[TM_W1], lw.w1, D, F, 64, 128) && make_tmap(&t[TM_W3], lw.w3, D, F, 64, 128) &&
+                 make_tmap(&t[TM_W2], lw.w2, F, D, 64, 128) && make_tmap(&t[TM_W1G], lw.w1, D, F, 64, 64) &&
+                 make_tmap(&t[TM_W3G], lw.w3, D, F, 64, 64);
         }
-        m->gemm_ok = ok;
+        if (ok && c.has_embed_and_head)
+            ok = make_tmap(&m->tm_head, c.tie_embeddings ? m->tok_emb : m->out, D, c.vocab, 64, 128);
+        if (ok) ok = make_tmap(&m->tm_hw, m->hw, D, Mx, 64, 128) && make_tmap(&m->tm_o, m->o, H * d, Mx, 64, 128) &&
+                     make_tmap(&m->tm_g, m->g, F, Mx, 64, 128);
+        if (!ok) return bail(fail(LLM_ERR_CUDA, "cuTensorMapEncodeTiled failed"));
+        m->gemm_ok = D % GEMM_BN == 0 && (H * d) % GEMM_BN == 0 && (Hk * d) % GEMM_BN == 0 &&
+                     F % (GEMM_BN / 2) == 0 && D % GEMM_BK == 0 && F % GEMM_BK == 0 && (H * d) % GEMM_BK == 0;
         if (d == 128) {
             const uint64_t rows = (uint64_t)c.n_layers * c.max_batch * Hk * c.max_seq_len;
             if (!make_tmap(&m->tm_kc, m->kc, d, rows, 64, 64) || !make_tmap(&m->tm_vc, m->vc, d, rows, 64, 64))
@@ -677,6 +745,7 @@ int llm_prefill(llm_model* m, const int32_t* tokens, int B, int T, int32_t* next
 
 int llm_prefill_hidden(llm_model* m, const float* h_in, int B, int T, float* h_out) {
     if (!m || !h_in || !h_out) return fail(LLM_ERR_NULL_PTR, "model, h_in or h_out is NULL");
+    if (!aligned16(h_in) || !aligned16(h_out)) return fail(LLM_ERR_BAD_ARG, "h_in and h_out must be 16-byte aligned");
     int rc = check_batch(m, B, T);
     if (rc) return rc;
     rc = run_embed(m, nullptr, h_in, B * T);
@@ -685,7 +754,7 @@ int llm_prefill_hidden(llm_model* m, const float* h_in, int B, int T, float* h_o
     if (rc) return rc;
     {
         KTimer timer(m, LLM_K_OUT);
-        CK(launch_finish_hidden(m->h, h_out, (long long)B * T * m->cfg.dim, m->seq_len, B, T, m->stream, true));
+        CK(launch_finish_hidden(m->h, h_out, (long long)B * T * m->cfg.dim, m->seq_len, B, T, m->stream, m->pdl));
     }
     for (int b = 0; b < B; ++b) m->host_len[b] += T;
     return LLM_OK;
@@ -706,6 +775,7 @@ int llm_decode_step(llm_model* m, int B, const int32_t* in_tok, int32_t* next, f
             cudaGraph_t graph = nullptr;
             CK(cudaStreamBeginCapture(m->stream, cudaStreamCaptureModeThreadLocal));
             m->capturing = true;
+            m->cap_recs.clear();
             rc = decode_core(m, B, m->d_tok, m->d_next, logits ? m->d_logits : nullptr);
             m->capturing = false;
             cudaError_t ec = cudaStreamEndCapture(m->stream, &graph);
@@ -718,10 +788,20 @@ int llm_decode_step(llm_model* m, int B, const int32_t* in_tok, int32_t* next, f
             ec = cudaGraphInstantiate(&exec, graph, 0);
             cudaGraphDestroy(graph);
             if (ec != cudaSuccess) return fail(LLM_ERR_CUDA, "graph instantiate: %s", cudaGetErrorString(ec));
-            it = m->graphs.emplace(key, exec).first;
+            it = m->graphs.emplace(key, llm_model::Graph{exec, m->cap_recs}).first;
+            m->cap_recs.clear();
         }
         CK(cudaMemcpyAsync(m->d_tok, in_tok, (size_t)B * 4, cudaMemcpyDeviceToDevice, m->stream));
-        CK(cudaGraphLaunch(it->second, m->stream));
+        CK(cudaGraphLaunch(it->second.exec, m->stream));
+        if (!it->second.recs.empty()) {  // timing: read this replay's event pairs
+            CK(cudaStreamSynchronize(m->stream));
+            for (const auto& r : it->second.recs) {
+                float ms = 0.f;
+                CK(cudaEventElapsedTime(&ms, r.a, r.b));
+                m->kt_ms[r.kind] += ms;
+                m->kt_n[r.kind] += 1;
+            }
+        }
         CK(cudaMemcpyAsync(next, m->d_next, (size_t)B * 4, cudaMemcpyDeviceToDevice, m->stream));
         if (logits)
             CK(cudaMemcpyAsync(logits, m->d_logits, (size_t)B * V * 4, cudaMemcpyDeviceToDevice, m->stream));
@@ -789,25 +869,24 @@ int llm_debug_tap(llm_model* m, int layer, float* dst, size_t dst_elems) {
 int llm_kernel_times(llm_model* m, int n, double* total_ms, int64_t* launches, int reset) {
     if (!m || (n > 0 && (!total_ms || !launches))) return fail(LLM_ERR_NULL_PTR, "NULL argument");
     CK(cudaStreamSynchronize(m->stream));
-    for (int i = 0; i < n; ++i) {
-        total_ms[i] = 0.0;
-        launches[i] = 0;
-    }
     for (const auto& r : m->trecs) {
         float ms = 0.f;
         CK(cudaEventElapsedTime(&ms, r.a, r.b));
-        if (r.kind < n) {
-            total_ms[r.kind] += ms;
-            launches[r.kind] += 1;
-        }
+        m->kt_ms[r.kind] += ms;
+        m->kt_n[r.kind] += 1;
+        m->ev_pool.push_back(r.a);
+        m->ev_pool.push_back(r.b);
     }
-    if (reset) {
-        for (const auto& r : m->trecs) {
-            m->ev_pool.push_back(r.a);
-            m->ev_pool.push_back(r.b);
-        }
-        m->trecs.clear();
+    m->trecs.clear();
+    for (int i = 0; i < n; ++i) {
+        total_ms[i] = i < LLM_K_COUNT ? m->kt_ms[i] : 0.0;
+        launches[i] = i < LLM_K_COUNT ? m->kt_n[i] : 0;
     }
+    if (reset)
+        for (int i = 0; i < LLM_K_COUNT; ++i) {
+            m->kt_ms[i] = 0.0;
+            m->kt_n[i] = 0;
+        }
     return LLM_OK;
 }
 
@@ -855,22 +934,61 @@ int llm_op_gemm_bf16(const void* A, const void* B, float* C, int M, int N, int K
     return LLM_OK;
 }
 
-int llm_op_gemv_bf16(const void* x, const void* W, float* y, int M, int N, int K, void* stream) {
-    if (!x || !W || !y) return fail(LLM_ERR_NULL_PTR, "NULL operand");
+// Workspace layout of the single-operation GEMV: [tile counters | packed maxima
+// | done counter | partial fragments], each part 256-byte aligned.
+static size_t gemv_ws_layout(int N, int K, size_t* off_part, GemvScratch* ws, void* base) {
+    const int sms = num_sms_current();
+    const int tiles = gemv_num_tiles(EPI_STORE_F32, N);
+    const size_t pf = gemv_scratch_floats(EPI_STORE_F32, N, K, sms);
+    const size_t o_cnt = 0;
+    const size_t o_best = (o_cnt + (size_t)tiles * 4 + 255) & ~size_t(255);
+    const size_t o_done = o_best + 256;
+    const size_t o_part = o_done + 256;
+    if (off_part) *off_part = o_part;
+    if (ws && base) {
+        char* b = reinterpret_cast<char*>(base);
+        ws->tile_cnt = reinterpret_cast<unsigned*>(b + o_cnt);
+        ws->tiles_cap = tiles;
+        ws->am_best = reinterpret_cast<unsigned long long*>(b + o_best);
+        ws->done_cnt = reinterpret_cast<unsigned*>(b + o_done);
+        ws->part = reinterpret_cast<float*>(b + o_part);
+        ws->part_floats = pf;
+    }
+    return o_part + pf * 4;
+}
+
+size_t llm_op_gemv_workspace(int N, int K) {
+    if (N < 1 || K < 8 || K % 8 != 0) return 0;
+    return gemv_ws_layout(N, K, nullptr, nullptr, nullptr);
+}
+
+int llm_op_gemv_bf16(const void* x, const void* W, float* y, int M, int N, int K, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+    if (!x || !W || !y || !workspace) return fail(LLM_ERR_NULL_PTR, "NULL operand or workspace");
     if (M < 1 || M > 16 || N < 1 || K < 8 || K % 8 != 0) return fail(LLM_ERR_BAD_ARG, "need 1 <= M <= 16, K %% 8 == 0");
-    if (!aligned16(x) || !aligned16(W)) return fail(LLM_ERR_BAD_ARG, "operands must be 16-byte aligned");
+    if (!aligned16(x) || !aligned16(W) || !aligned16(workspace))
+        return fail(LLM_ERR_BAD_ARG, "operands must be 16-byte aligned");
     GemvArgs<__nv_bfloat16> ga;
+    size_t off_part = 0;
+    if (workspace_bytes < gemv_ws_layout(N, K, &off_part, &ga.ws, workspace))
+        return fail(LLM_ERR_BAD_ARG, "workspace too small");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    CK(cudaMemsetAsync(workspace, 0, off_part, s));
+    CUtensorMap tw;
+    if (!make_tmap(&tw, W, K, N, 64, 128)) return fail(LLM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    ga.tmw[0] = &tw;
     ga.W[0] = reinterpret_cast<const __nv_bfloat16*>(W);
     ga.N = N;
     ga.K = K;
     ga.x = reinterpret_cast<const __nv_bfloat16*>(x);
     ga.ldx = K;
     ga.M = M;
+    ga.num_sms = num_sms_current();
     ga.epi.kind = EPI_STORE_F32;
     ga.epi.M = M;
     ga.epi.y = y;
     ga.epi.ldy = N;
-    CK(launch_gemv_bf16(ga, reinterpret_cast<cudaStream_t>(stream), false));
+    CK(launch_gemv_bf16(ga, s, false));
     return LLM_OK;
 }
 
@@ -948,6 +1066,7 @@ int llm_op_attention_decode(const void* q, const void* kcache, const void* vcach
     a.ws_part = reinterpret_cast<float*>(workspace);
     a.ws_count = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(workspace) + part_bytes);
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
+    a.err = op_err_ptr();
     CK(cudaMemsetAsync(a.ws_count, 0, p.counters * 4, s));
     CK(launch_attn_decode(a, dtype == LLM_BF16, s, false));
     return LLM_OK;

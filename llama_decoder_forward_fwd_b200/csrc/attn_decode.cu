@@ -9,12 +9,15 @@
 // A CTA owns one (sequence, KV head, chunk of query tokens) and one contiguous
 // slice ("split") of the keys; its rows are the G query heads of the KV head for
 // each query token, so each key and value row is read once for the whole group.
-// Lane j of a warp scores key j of a 32-key group for every row, the warp keeps
-// an online softmax (running max and sum, log2 domain), and accumulates
-// P V with lane l owning dims 4l..4l+3. The 4 warps' states and then the splits'
-// states (m, l, o) are merged by the log-sum-exp rule; the merge across
-// splits is done by whichever CTA of the (sequence, head, chunk) finishes last
-// (an atomic counter, no waiting), which also resets the counter.
+// Each of the 4 warps takes 32-key groups of the split. Lane j loads the whole
+// key row j into registers and the value slice (dims 4l..4l+3) of all 32 keys,
+// every load issued before the first use, so a group costs one memory round
+// trip. Lane j scores key j for every row against the query rows, which all
+// lanes read from shared memory as broadcasts; the warp keeps an online softmax
+// (running max and sum, log2 domain) and accumulates P V. The warps' states,
+// then the splits' states (m, l, o), are merged by the log-sum-exp rule; the
+// split merge is done by whichever CTA of the group finishes last (an atomic
+// counter, no waiting), which also resets the counter.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -23,36 +26,45 @@
 namespace lfw {
 
 constexpr int AD_THREADS = 128;
+constexpr int AD_WARPS = 4;
+constexpr int AD_GK = 32;     // keys per group (one per lane)
 constexpr int AD_DMAX = 128;
+constexpr int AD_MAX_SPLITS = 64;
 
-template <typename KT> DEVI void load8(const KT* p, float (&v)[8]);
-template <> DEVI void load8<float>(const float* p, float (&v)[8]) {
-    const float4 a = reinterpret_cast<const float4*>(p)[0];
-    const float4 b = reinterpret_cast<const float4*>(p)[1];
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+template <typename KT> DEVI void unpack16(const uint4& u, float (&v)[16 / sizeof(KT)]);
+template <> DEVI void unpack16<float>(const uint4& u, float (&v)[4]) {
+    v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y); v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
 }
-template <> DEVI void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8]) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
+template <> DEVI void unpack16<__nv_bfloat16>(const uint4& u, float (&v)[8]) {
     v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
     v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
 }
-template <typename KT> DEVI void load4(const KT* p, float (&v)[4]);
-template <> DEVI void load4<float>(const float* p, float (&v)[4]) {
-    const float4 a = *reinterpret_cast<const float4*>(p);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+// Four consecutive elements as raw bits (8 bytes of bf16 or 16 bytes of fp32).
+template <typename KT> struct Vec4;
+template <> struct Vec4<float> { using T = uint4; };
+template <> struct Vec4<__nv_bfloat16> { using T = uint2; };
+DEVI void to4(const uint4& u, float (&v)[4]) {
+    v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y); v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
 }
-template <> DEVI void load4<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[4]) {
-    const uint2 u = *reinterpret_cast<const uint2*>(p);
-    v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
-}
+DEVI void to4(const uint2& u, float (&v)[4]) { v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y); }
 
 template <typename KT, int RMAX>
 __global__ void __launch_bounds__(AD_THREADS) attn_decode_kernel(const AttnDecodeArgs a) {
-    __shared__ __align__(16) float qs[RMAX][AD_DMAX];
-    __shared__ float wm[4][RMAX], wl[4][RMAX];
-    __shared__ __align__(16) float wo[4][RMAX][AD_DMAX];
+    constexpr int EPC = 16 / sizeof(KT);  // elements per 16-byte chunk
+    constexpr int NCH = AD_DMAX / EPC;    // chunks of a full-width key row
+    constexpr int KBATCH = NCH < 16 ? NCH : 16;                 // key-row chunks loaded together
+    constexpr int VBATCH = sizeof(KT) == 2 ? AD_GK : AD_GK / 2;  // value rows loaded together
+    using V4 = typename Vec4<KT>::T;
+    // qs (query rows * log2(e)/sqrt(d)) during the keys, then the split weights
+    // and sums sm_m/sm_l [RMAX][64] each during the split merge.
+    __shared__ __align__(16) float qbuf[RMAX * AD_DMAX];
+    __shared__ float wm[AD_WARPS][RMAX], wl[AD_WARPS][RMAX];
+    __shared__ __align__(16) float wo[AD_WARPS][RMAX][AD_DMAX];
     __shared__ int last_s;
+    float(*qs)[AD_DMAX] = reinterpret_cast<float(*)[AD_DMAX]>(qbuf);
+    float(*sm_m)[AD_MAX_SPLITS] = reinterpret_cast<float(*)[AD_MAX_SPLITS]>(qbuf);
+    float(*sm_l)[AD_MAX_SPLITS] = reinterpret_cast<float(*)[AD_MAX_SPLITS]>(qbuf + RMAX * AD_MAX_SPLITS);
+    static_assert(2 * AD_MAX_SPLITS <= AD_DMAX, "split merge scratch must fit in the query buffer");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int split = blockIdx.x, qc = blockIdx.z;
@@ -60,6 +72,7 @@ __global__ void __launch_bounds__(AD_THREADS) attn_decode_kernel(const AttnDecod
     const int G = a.H / a.Hk, d = a.d;
     const int R = a.tq * G;
     const int HD = a.H * d;
+    const int nch = d / EPC;
     const KT* q = reinterpret_cast<const KT*>(a.q);
     const long long head_off = (long long)(b * a.Hk + kvh) * a.S_max * d;
     const KT* kc = reinterpret_cast<const KT*>(a.kc) + head_off;
@@ -73,20 +86,37 @@ __global__ void __launch_bounds__(AD_THREADS) attn_decode_kernel(const AttnDecod
     // keys [0, limit) are visible to some row; never read past the cache
     const int limit = min(p0 + t_last + 1, a.S_max);
     int chunk = (limit + a.n_splits - 1) / a.n_splits;
-    chunk = (chunk + 31) & ~31;
+    chunk = (chunk + AD_GK - 1) & ~(AD_GK - 1);
     const int kbeg = split * chunk;
     const int kend = min(limit, kbeg + chunk);
 
-    // Query rows, pre-scaled by log2(e)/sqrt(d).
-    for (int idx = threadIdx.x; idx < RMAX * AD_DMAX; idx += AD_THREADS) {
-        const int r = idx / AD_DMAX, dd = idx % AD_DMAX;
-        float v = 0.f;
-        const int t = t_first + r / G;
-        if (r < R && t < a.T && dd < d) {
-            const int h = kvh * G + r % G;
-            v = to_f<KT>(q[(long long)(b * a.T + t) * HD + h * d + dd]) * a.scale_log2;
+    // The first key-row batch and value batch of this warp's first group are
+    // requested now, so their latency overlaps the query staging below.
+    const bool own_dims = 4 * lane < d;
+    uint4 kr0[KBATCH];
+    V4 vr0[VBATCH];
+    auto load_first = [&](int kb) {
+        const int jj0 = kb + lane;
+        const uint4* kp = reinterpret_cast<const uint4*>(kc + (long long)(jj0 < kend ? jj0 : kb) * d);
+#pragma unroll
+        for (int c = 0; c < KBATCH; ++c) kr0[c] = (c < nch && kb < kend) ? kp[c] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int jj = 0; jj < VBATCH; ++jj) {
+            if (kb + jj < kend && own_dims) vr0[jj] = *reinterpret_cast<const V4*>(vc + (long long)(kb + jj) * d + 4 * lane);
+            else vr0[jj] = V4{};
         }
-        qs[r][dd] = v;
+    };
+    load_first(kbeg + warp * AD_GK);
+
+    // Query rows, pre-scaled by log2(e)/sqrt(d): 4 elements per thread per step.
+    for (int idx = threadIdx.x; idx < RMAX * (AD_DMAX / 4); idx += AD_THREADS) {
+        const int r = idx / (AD_DMAX / 4), dd = (idx % (AD_DMAX / 4)) * 4;
+        float v[4] = {0.f, 0.f, 0.f, 0.f};
+        const int t = t_first + r / G;
+        if (r < R && t < a.T && dd < d)
+            to4(*reinterpret_cast<const V4*>(q + (long long)(b * a.T + t) * HD + (kvh * G + r % G) * d + dd), v);
+        *reinterpret_cast<float4*>(&qs[r][dd]) =
+            make_float4(v[0] * a.scale_log2, v[1] * a.scale_log2, v[2] * a.scale_log2, v[3] * a.scale_log2);
     }
     int plim[RMAX];  // last visible key of each row (-1: no row)
 #pragma unroll
@@ -103,25 +133,37 @@ __global__ void __launch_bounds__(AD_THREADS) attn_decode_kernel(const AttnDecod
         l[r] = 0.f;
         o[r][0] = o[r][1] = o[r][2] = o[r][3] = 0.f;
     }
-    const bool own_dims = 4 * lane < d;
 
-    for (int kb = kbeg + warp * 32; kb < kend; kb += 4 * 32) {
+    for (int kb = kbeg + warp * AD_GK; kb < kend; kb += AD_WARPS * AD_GK) {
         const int j = kb + lane;
         const bool jv = j < kend;
+        const int nk = min(AD_GK, kend - kb);
+        // This lane's key row, KBATCH 16-byte chunks per batch with every load of a
+        // batch issued before its first use (one batch for bf16 rows).
+        const uint4* kp = reinterpret_cast<const uint4*>(kc + (long long)(jv ? j : kb) * d);
         float s[RMAX];
 #pragma unroll
         for (int r = 0; r < RMAX; ++r) s[r] = 0.f;
-        if (jv) {
-            const KT* kp = kc + (long long)j * d;
-            for (int dd = 0; dd < d; dd += 8) {
-                float kv[8];
-                load8<KT>(kp + dd, kv);
 #pragma unroll
-                for (int r = 0; r < RMAX; ++r) {
-                    const float4 qa = *reinterpret_cast<const float4*>(&qs[r][dd]);
-                    const float4 qb = *reinterpret_cast<const float4*>(&qs[r][dd + 4]);
-                    s[r] += qa.x * kv[0] + qa.y * kv[1] + qa.z * kv[2] + qa.w * kv[3] + qb.x * kv[4] +
-                            qb.y * kv[5] + qb.z * kv[6] + qb.w * kv[7];
+        for (int c0 = 0; c0 < NCH; c0 += KBATCH) {
+            if (c0 >= nch) break;
+            uint4 kr[KBATCH];
+#pragma unroll
+            for (int c = 0; c < KBATCH; ++c)
+                kr[c] = c0 == 0 ? kr0[c] : ((c0 + c < nch) ? kp[c0 + c] : make_uint4(0, 0, 0, 0));
+#pragma unroll
+            for (int c = 0; c < KBATCH; ++c) {
+                if (c0 + c < nch) {
+                    float kv[EPC];
+                    unpack16<KT>(kr[c], kv);
+#pragma unroll
+                    for (int r = 0; r < RMAX; ++r) {
+#pragma unroll
+                        for (int e = 0; e < EPC; e += 4) {
+                            const float4 qv = *reinterpret_cast<const float4*>(&qs[r][(c0 + c) * EPC + e]);  // broadcast
+                            s[r] += qv.x * kv[e] + qv.y * kv[e + 1] + qv.z * kv[e + 2] + qv.w * kv[e + 3];
+                        }
+                    }
                 }
             }
         }
@@ -137,19 +179,34 @@ __global__ void __launch_bounds__(AD_THREADS) attn_decode_kernel(const AttnDecod
             l[r] = l[r] * alpha + warp_sum(p[r]);
             m[r] = mnew;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) o[r][i] *= alpha;
+            for (int e = 0; e < 4; ++e) o[r][e] *= alpha;
         }
-        const int nv = min(32, kend - kb);
-        for (int jj = 0; jj < nv; ++jj) {
-            float vv[4] = {0.f, 0.f, 0.f, 0.f};
-            if (own_dims) load4<KT>(vc + (long long)(kb + jj) * d + 4 * lane, vv);
+        // Value slices of VBATCH keys per batch, all loads of a batch issued first.
 #pragma unroll
-            for (int r = 0; r < RMAX; ++r) {
-                const float pj = __shfl_sync(0xffffffffu, p[r], jj);
+        for (int j0 = 0; j0 < AD_GK; j0 += VBATCH) {
+            V4 vr[VBATCH];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) o[r][i] += pj * vv[i];
+            for (int jj = 0; jj < VBATCH; ++jj) {
+                if (j0 == 0)
+                    vr[jj] = vr0[jj];
+                else if (j0 + jj < nk && own_dims)
+                    vr[jj] = *reinterpret_cast<const V4*>(vc + (long long)(kb + j0 + jj) * d + 4 * lane);
+                else
+                    vr[jj] = V4{};
+            }
+#pragma unroll
+            for (int jj = 0; jj < VBATCH; ++jj) {
+                float vv[4];
+                to4(vr[jj], vv);
+#pragma unroll
+                for (int r = 0; r < RMAX; ++r) {
+                    const float pj = __shfl_sync(0xffffffffu, p[r], j0 + jj);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o[r][e] += pj * vv[e];
+                }
             }
         }
+        if (kb + AD_WARPS * AD_GK < kend) load_first(kb + AD_WARPS * AD_GK);
     }
 
     // Merge the 4 warps.
@@ -162,22 +219,22 @@ __global__ void __launch_bounds__(AD_THREADS) attn_decode_kernel(const AttnDecod
         if (own_dims) *reinterpret_cast<float4*>(&wo[warp][r][4 * lane]) = make_float4(o[r][0], o[r][1], o[r][2], o[r][3]);
     }
     __syncthreads();
-    const long long rec = d + 2;
+    const long long rec = d + 4;  // m, l, 2 pad, o[d]: o starts 16-byte aligned
     const long long grp = ((long long)(b * a.Hk + kvh) * a.n_qchunks + qc);
     float* part = a.ws_part + grp * R * a.n_splits * rec;
     for (int idx = threadIdx.x; idx < R * d; idx += AD_THREADS) {
         const int r = idx / d, dd = idx % d;
         float M = -INFINITY;
-        for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w][r]);
+        for (int w = 0; w < AD_WARPS; ++w) M = fmaxf(M, wm[w][r]);
         const float Mu = (M == -INFINITY) ? 0.f : M;
         float L = 0.f, O = 0.f;
-        for (int w = 0; w < 4; ++w) {
+        for (int w = 0; w < AD_WARPS; ++w) {
             const float sc = exp2f(wm[w][r] - Mu);
             L += sc * wl[w][r];
             O += sc * wo[w][r][dd];
         }
         float* pr = part + ((long long)r * a.n_splits + split) * rec;
-        pr[2 + dd] = O;
+        pr[4 + dd] = O;
         if (dd == 0) {
             pr[0] = M;
             pr[1] = L;
@@ -194,22 +251,54 @@ __global__ void __launch_bounds__(AD_THREADS) attn_decode_kernel(const AttnDecod
     __syncthreads();
     if (!last_s) return;
     __threadfence();
-    KT* out = reinterpret_cast<KT*>(a.out);
-    for (int idx = threadIdx.x; idx < R * d; idx += AD_THREADS) {
-        const int r = idx / d, dd = idx % d;
-        const int t = t_first + r / G;
-        if (t >= a.T) continue;
-        const int h = kvh * G + r % G;
-        const float* pr = part + (long long)r * a.n_splits * rec;
+    const int ns = a.n_splits;
+    for (int idx = threadIdx.x; idx < R * ns; idx += AD_THREADS) {
+        const int r = idx / ns, sp = idx % ns;
+        const float* pr = part + ((long long)r * ns + sp) * rec;
+        sm_m[r][sp] = __ldcg(pr);
+        sm_l[r][sp] = __ldcg(pr + 1);
+    }
+    __syncthreads();
+    // Split weights w_s = exp2(m_s - max) / sum_s exp2(m_s - max) l_s, kept in sm_m.
+    for (int r = threadIdx.x; r < R; r += AD_THREADS) {
         float M = -INFINITY;
-        for (int sp = 0; sp < a.n_splits; ++sp) M = fmaxf(M, __ldcg(pr + sp * rec));
-        float L = 0.f, O = 0.f;
-        for (int sp = 0; sp < a.n_splits; ++sp) {
-            const float sc = exp2f(__ldcg(pr + sp * rec) - M);
-            L += sc * __ldcg(pr + sp * rec + 1);
-            O += sc * __ldcg(pr + sp * rec + 2 + dd);
+        for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, sm_m[r][sp]);
+        const float Mu = (M == -INFINITY) ? 0.f : M;
+        float L = 0.f;
+        for (int sp = 0; sp < ns; ++sp) {
+            const float w = exp2f(sm_m[r][sp] - Mu);
+            sm_m[r][sp] = w;
+            L += w * sm_l[r][sp];
         }
-        out[(long long)(b * a.T + t) * HD + h * d + dd] = from_f<KT>(O / L);
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        for (int sp = 0; sp < ns; ++sp) sm_m[r][sp] *= inv;
+    }
+    __syncthreads();
+    // Each thread owns (row, 4 dims) outputs and sums the weighted splits; the
+    // loads of different splits are independent, so they overlap.
+    KT* out = reinterpret_cast<KT*>(a.out);
+    const int dq = d / 4;
+    for (int idx = threadIdx.x; idx < R * dq; idx += AD_THREADS) {
+        const int r = idx / dq, d4 = (idx % dq) * 4;
+        const float* pr = part + (long long)r * ns * rec + 4 + d4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int sp = 0; sp < ns; ++sp) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(pr + (long long)sp * rec));
+            const float w = sm_m[r][sp];
+            acc.x += w * v.x;
+            acc.y += w * v.y;
+            acc.z += w * v.z;
+            acc.w += w * v.w;
+        }
+        const int t = t_first + r / G;
+        if (t < a.T) {
+            KT* dst = out + (long long)(b * a.T + t) * HD + (kvh * G + r % G) * d + d4;
+            dst[0] = from_f<KT>(acc.x);
+            dst[1] = from_f<KT>(acc.y);
+            dst[2] = from_f<KT>(acc.z);
+            dst[3] = from_f<KT>(acc.w);
+        }
     }
     if (threadIdx.x == 0) a.ws_count[grp] = 0u;
 }
@@ -221,30 +310,43 @@ AttnDecodePlan attn_decode_plan(int B, int T, int H, int Hk, int d, int max_keys
     if (p.tq < 1) p.tq = 1;
     p.n_qchunks = (T + p.tq - 1) / p.tq;
     const int groups = B * Hk * p.n_qchunks;
-    int ns = (2 * num_sms + groups - 1) / groups;
+    // About 128 keys per CTA (one 32-key group per warp), at least one CTA per SM,
+    // at least 32 keys per split.
     const int by_len = (max_keys + 127) / 128;
-    if (ns > by_len) ns = by_len;
-    if (ns > 64) ns = 64;
+    const int fill = (num_sms + groups - 1) / groups;
+    const int cap = (max_keys + AD_GK - 1) / AD_GK;
+    int ns = by_len > fill ? by_len : fill;
+    if (ns > cap) ns = cap;
+    if (ns > AD_MAX_SPLITS) ns = AD_MAX_SPLITS;
     if (ns < 1) ns = 1;
     p.n_splits = ns;
-    p.part_floats = (size_t)groups * p.tq * G * ns * (d + 2);
+    p.part_floats = (size_t)groups * p.tq * G * ns * (d + 4);
     p.counters = groups;
     return p;
+}
+
+template <typename KT, int RMAX>
+static cudaError_t launch_one(const AttnDecodeArgs& a, cudaStream_t s, bool pdl) {
+    const dim3 grid(a.n_splits, a.B * a.Hk, a.n_qchunks);
+    return launch_k(attn_decode_kernel<KT, RMAX>, grid, AD_THREADS, 0, s, pdl, a);
 }
 
 cudaError_t launch_attn_decode(const AttnDecodeArgs& a, bool bf16, cudaStream_t s, bool pdl) {
     const int G = a.H / a.Hk;
     const int R = a.tq * G;
-    if (a.H % a.Hk != 0 || R > 16 || a.d > AD_DMAX || a.d % 8 != 0) return cudaErrorInvalidValue;
-    const dim3 grid(a.n_splits, a.B * a.Hk, a.n_qchunks);
+    if (a.H % a.Hk != 0 || R > 16 || a.d > AD_DMAX || a.d % 8 != 0 || a.n_splits > AD_MAX_SPLITS)
+        return cudaErrorInvalidValue;
     if (bf16) {
-        if (R <= 4) return launch_k(attn_decode_kernel<__nv_bfloat16, 4>, grid, AD_THREADS, 0, s, pdl, a);
-        if (R <= 8) return launch_k(attn_decode_kernel<__nv_bfloat16, 8>, grid, AD_THREADS, 0, s, pdl, a);
-        return launch_k(attn_decode_kernel<__nv_bfloat16, 16>, grid, AD_THREADS, 0, s, pdl, a);
+        if (R <= 4) return launch_one<__nv_bfloat16, 4>(a, s, pdl);
+        if (R <= 8) return launch_one<__nv_bfloat16, 8>(a, s, pdl);
+        return launch_one<__nv_bfloat16, 16>(a, s, pdl);
     }
-    if (R <= 4) return launch_k(attn_decode_kernel<float, 4>, grid, AD_THREADS, 0, s, pdl, a);
-    if (R <= 8) return launch_k(attn_decode_kernel<float, 8>, grid, AD_THREADS, 0, s, pdl, a);
-    return launch_k(attn_decode_kernel<float, 16>, grid, AD_THREADS, 0, s, pdl, a);
+    if (R <= 4) return launch_one<float, 4>(a, s, pdl);
+    if (R <= 8) return launch_one<float, 8>(a, s, pdl);
+    return launch_one<float, 16>(a, s, pdl);
 }
+
+// Nothing to configure: the kernel uses static shared memory only.
+cudaError_t attn_decode_prepare() { return cudaSuccess; }
 
 }  // namespace lfw

@@ -20,6 +20,8 @@ enum : uint32_t {
     DERR_GEMM_MMA_WAIT = 0x102,
     DERR_GEMM_EPI_WAIT = 0x103,
     DERR_ATTN_TMA_WAIT = 0x201,
+    DERR_GEMV_PRODUCER_WAIT = 0x301,
+    DERR_GEMV_CONSUMER_WAIT = 0x302,
 };
 
 // 4 seconds: far longer than any legitimate wait for one pipeline stage.
@@ -39,6 +41,9 @@ DEVI uint64_t globaltimer() {
 DEVI void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // pdl_trigger(): allow the next kernel in the stream to start launching.
 DEVI void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Barrier over the first `count` threads of the CTA (id 1..15; 0 is __syncthreads).
+DEVI void named_bar_sync(int id, int count) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory"); }
 
 // ---- mbarrier ---------------------------------------------------------
 DEVI void mbar_init(uint64_t* bar, uint32_t count) {
@@ -92,6 +97,14 @@ DEVI void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
             smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+// Untiled bulk copy global -> shared (both 16-byte aligned, bytes % 16 == 0).
+DEVI void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
 

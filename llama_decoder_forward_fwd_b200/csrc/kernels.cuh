@@ -76,6 +76,24 @@ struct Epi {
 };
 
 // ---- decode projection: y = x W^T for M <= 16 token rows ---------------
+// Device scratch of the streaming bf16 GEMV. Counters and packed maxima must be
+// zero before the first launch; every launch leaves them zero again.
+struct GemvScratch {
+    float* part = nullptr;                  // partial fragments of split tiles
+    size_t part_floats = 0;
+    unsigned* tile_cnt = nullptr;           // [tiles_cap] k blocks finished per tile
+    int tiles_cap = 0;
+    unsigned long long* am_best = nullptr;  // [16] packed (logit, id) maxima
+    unsigned* done_cnt = nullptr;           // [1] tiles finished (argmax)
+};
+struct GemvPlan {
+    int ntiles, nkb, grid, max_pieces;
+    long long TB;
+};
+GemvPlan gemv_plan(int kind, int N, int K, int num_sms, int occ);
+// Partial-buffer floats any launch of this shape can need.
+size_t gemv_scratch_floats(int kind, int N, int K, int num_sms);
+
 template <typename T>
 struct GemvArgs {
     const T* W[3] = {nullptr, nullptr, nullptr};  // QKV: wq, wk, wv; SWIGLU: w1, w3; else W[0]
@@ -86,10 +104,16 @@ struct GemvArgs {
     int ldx = 0;
     int M = 0;   // rows in this launch (<= 16)
     int m0 = 0;  // token index of row 0 (the epilogue sees token m0 + m)
+    int num_sms = 148;
+    GemvScratch ws;                                           // bf16 kernel only
+    const CUtensorMap* tmw[3] = {nullptr, nullptr, nullptr};  // bf16 kernel: box 64 x 128 rows
+                                                              // (SwiGLU: w1, w3 with 64-row boxes)
     Epi epi;
 };
-// Number of 16-row tiles (parts of the RESID partial sums, tiles of LOGITS partials).
+// Row tiles of the bf16 decode projection (128 rows; 64 w1 + 64 w3 rows for SwiGLU).
 int gemv_num_tiles(int kind, int N);
+// Parts of the RMSNorm partial sums a projection with N output rows writes (one per 16 rows).
+inline int gemv_ss_parts(int N) { return (N + 15) / 16; }
 cudaError_t launch_gemv_bf16(const GemvArgs<__nv_bfloat16>& a, cudaStream_t s, bool pdl);
 cudaError_t launch_gemv_f32(const GemvArgs<float>& a, cudaStream_t s, bool pdl);
 
@@ -131,6 +155,7 @@ struct AttnDecodeArgs {
     float* ws_part = nullptr;       // split partials (m, l, o[d])
     unsigned* ws_count = nullptr;   // [B*Hk*n_qchunks], zero between launches
     float scale_log2 = 0.f;
+    uint32_t* err = nullptr;
 };
 struct AttnDecodePlan {
     int n_splits, tq, n_qchunks;
@@ -138,6 +163,7 @@ struct AttnDecodePlan {
 };
 AttnDecodePlan attn_decode_plan(int B, int T, int H, int Hk, int d, int max_keys, int num_sms);
 cudaError_t launch_attn_decode(const AttnDecodeArgs& a, bool bf16, cudaStream_t s, bool pdl);
+cudaError_t attn_decode_prepare();
 
 // ---- small kernels ----------------------------------------------------
 struct EmbedArgs {

@@ -10,7 +10,9 @@ constexpr int EMB_THREADS = 256;
 
 // h[m] = E[tok[m]] ("Building llama3 from scratch": the embedding layer maps each
 // token id to its row of tok_embeddings) or the given hidden state, plus the first
-// layer's RMSNorm inputs: hw[m] = h[m] * w and ss[m] = sum h[m]^2.
+// layer's RMSNorm inputs: hw[m] = h[m] * w and ss[m] = sum h[m]^2. Each thread
+// moves 8 consecutive elements per step with 16-byte accesses, so a row costs one
+// memory round trip.
 template <typename WT>
 __global__ void __launch_bounds__(EMB_THREADS) embed_kernel(const EmbedArgs a) {
     __shared__ float red[EMB_THREADS / 32];
@@ -30,11 +32,25 @@ __global__ void __launch_bounds__(EMB_THREADS) embed_kernel(const EmbedArgs a) {
         src = reinterpret_cast<const WT*>(a.E) + (long long)tok * a.D;
     }
     float ss = 0.f;
-    for (int i = threadIdx.x; i < a.D; i += EMB_THREADS) {
-        const float v = hsrc ? hsrc[i] : to_f<WT>(src[i]);
-        h[i] = v;
-        hw[i] = from_f<WT>(v * to_f<WT>(wn[i]));
-        ss += v * v;
+    for (int i = threadIdx.x * 8; i < a.D; i += EMB_THREADS * 8) {  // D % 8 == 0
+        float v[8], w[8];
+        if (hsrc) {
+            const float4 x0 = *reinterpret_cast<const float4*>(hsrc + i);
+            const float4 x1 = *reinterpret_cast<const float4*>(hsrc + i + 4);
+            v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w; v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = to_f<WT>(src[i + j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w[j] = to_f<WT>(wn[i + j]);
+        reinterpret_cast<float4*>(h + i)[0] = make_float4(v[0], v[1], v[2], v[3]);
+        reinterpret_cast<float4*>(h + i)[1] = make_float4(v[4], v[5], v[6], v[7]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            hw[i + j] = from_f<WT>(v[j] * w[j]);
+            ss += v[j] * v[j];
+        }
     }
     ss = warp_sum(ss);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;

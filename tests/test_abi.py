@@ -83,6 +83,6 @@ def test_op_shape_checks_are_host_side(lib):
     p = ctypes.c_void_p(16)  # never dereferenced: the shape check fails first
     assert lib.llm_op_gemm_bf16(p, p, p, 4, 100, 64, None) == L.LLM_ERR_BAD_ARG     # N % 256
     assert lib.llm_op_gemm_bf16(p, p, p, 4, 256, 60, None) == L.LLM_ERR_BAD_ARG     # K % 64
-    assert lib.llm_op_gemv_bf16(p, p, p, 17, 16, 64, None) == L.LLM_ERR_BAD_ARG     # M > 16
+    assert lib.llm_op_gemv_bf16(p, p, p, 17, 16, 64, p, 1 << 20, None) == L.LLM_ERR_BAD_ARG  # M > 16
     assert lib.llm_op_attention_decode_workspace(1, 1, 32, 8, 128) > 0
     assert lib.llm_op_attention_decode_workspace(1, 1, 30, 8, 128) == 0             # H % Hk

@@ -49,7 +49,9 @@ def test_gemv_matches_definition(lib, M, N, K):
     x = _rand((M, K), torch.bfloat16, 3).to(DEV)
     W = _rand((N, K), torch.bfloat16, 4, 0.02).to(DEV)
     y = torch.full((M, N), float("nan"), device=DEV)
-    L.llm_op_gemv_bf16(x, W, y)
+    ws = torch.full((L.llm_op_gemv_workspace(N, K),), 255, dtype=torch.uint8, device=DEV)
+    for _ in range(2):  # the second call reuses the workspace the first left behind
+        L.llm_op_gemv_bf16(x, W, y, ws)
     torch.cuda.synchronize()
     _proj_check(x.cpu(), W.cpu(), y.cpu())
 
