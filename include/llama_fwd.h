@@ -261,6 +261,31 @@ int llm_op_attention_decode(const void* q, const void* kcache, const void* vcach
                             int d, int S_max, int dtype, void* workspace,
                             size_t workspace_bytes, void* stream);
 
+/*
+ * The split-KV decode attention of llm_op_attention_decode, for callers that
+ * cannot allocate device memory: code running while a stream is captured into
+ * a CUDA graph (cudaMalloc cannot be captured), plug-ins whose host
+ * application owns every device allocation, and latency-critical loops where
+ * an allocation could synchronise the device. The pages have no counterpart:
+ * this is a deployment convenience, not a step of the decoder.
+ *   Same arguments and results as llm_op_attention_decode, without the
+ *   workspace: the scratch is a fixed array inside the library (8 MiB of
+ *   per-split partial results and 4096 merge counters), held by every GPU that
+ *   loads the library until the process exits. The call allocates nothing
+ *   (no cudaMalloc, cudaFree or allocating library routine).
+ *   Shapes that need more scratch than that return LLM_ERR_BAD_ARG before
+ *   anything is queued (at B = 1..7 with 32 query heads, 8 KV heads and
+ *   head_dim 128 they fit).
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   Every call uses the same array and zeroes its counters first, so calls
+ *   whose kernels may overlap on the GPU (other streams, other host threads)
+ *   race with each other and must not be issued.
+ */
+int llm_op_attention_decode_static(const void* q, const void* kcache, const void* vcache,
+                                   const int32_t* pos0, void* out, int B, int T, int H, int Hk,
+                                   int d, int S_max, int dtype, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -78,6 +78,7 @@ _SIGS = {
     "llm_op_attention_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "llm_op_attention_decode_workspace": (_sz, [_i, _i, _i, _i, _i]),
     "llm_op_attention_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
+    "llm_op_attention_decode_static": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
 }
 
 
@@ -301,3 +302,11 @@ class Model:
             self.free()
         except Exception:
             pass
+
+
+def llm_op_attention_decode_static(q, kc, vc, pos0, out, stream=None):
+    """As llm_op_attention_decode, on the library's fixed scratch (no workspace, no allocation)."""
+    B, T, H, d = q.shape
+    Hk, S = kc.shape[1], kc.shape[2]
+    check(load().llm_op_attention_decode_static(_ptr(q), _ptr(kc), _ptr(vc), _ptr(pos0), _ptr(out), B, T, H, Hk, d,
+                                                S, _dt(q), _stream_ptr(stream)))

@@ -101,6 +101,8 @@ __device__ uint32_t g_op_err;  // device error word of the single-operation entr
 
 }  // namespace
 
+int lfw::set_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
 struct llm_model {
     llm_config cfg;
     int dev = 0, num_sms = 148;

@@ -183,6 +183,9 @@ cudaError_t launch_finish_hidden(const float* h, float* h_out, long long n, int3
 cudaError_t launch_rope_tables(float* cosv, float* sinv, int n_pos, int half, double theta, int head_dim,
                                cudaStream_t s);
 
+// Record msg as the calling thread's last error (llm_last_error) and return code.
+int set_error(int code, const char* msg);
+
 // Launch helper: programmatic stream serialization when pdl is set.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
