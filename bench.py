@@ -54,6 +54,7 @@ def work_model(shape, B, T, S_decode_mean):
     kinds_bytes = {  # one decode launch, B rows
         "qkv": 2 * D * (H + 2 * Hk) * d, "wo": 2 * H * d * D, "w13": 2 * 2 * F * D, "w2": 2 * F * D,
         "head": 2 * V * D, "attn": B * 2 * Hk * d * 2 * S_decode_mean,
+        "step": w_bytes + kv_bytes,  # the fused decode step: every weight and the cache, once
     }
     kinds_flops = {"qkv": 2 * B * T * D * (H + 2 * Hk) * d, "wo": 2 * B * T * H * d * D, "w13": 2 * B * T * 2 * F * D,
                    "w2": 2 * B * T * F * D, "attn": B * 4 * H * d * T * T / 2}
@@ -231,8 +232,9 @@ def run_ours(args, rank, world, local_rank):
 
     glob, layers = S.make_weights(shape, w.seed, device=dev)
     stream = torch.cuda.Stream(device=dev)
+    extra = L.LLM_FLAG_LAYERWISE_DECODE if args.layerwise else 0
     model = L.Model(shape, glob, layers, max_batch=B, max_tokens=B * T,
-                    flags=0 if args.no_graph else L.LLM_FLAG_CUDA_GRAPH, stream=stream, device=dev)
+                    flags=extra | (0 if args.no_graph else L.LLM_FLAG_CUDA_GRAPH), stream=stream, device=dev)
     prompt = S.make_tokens(w.seed, B, T, shape.vocab).to(dev)
     gen = torch.zeros(G + 1, B, dtype=torch.int32, device=dev)
 
@@ -319,7 +321,7 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- per-kernel CUDA-event timing of one step (roofline of the dominant kernel) ----
     tm = L.Model(shape, model.glob, model.layers, max_batch=B, max_tokens=B * T,
-                 flags=L.LLM_FLAG_KERNEL_TIMING | L.LLM_FLAG_CUDA_GRAPH, stream=stream, device=dev)
+                 flags=extra | L.LLM_FLAG_KERNEL_TIMING | L.LLM_FLAG_CUDA_GRAPH, stream=stream, device=dev)
     gen2 = torch.zeros_like(gen)
     L.llm_prefill(tm.h, prompt, gen2[0])
     kt_pre = L.llm_kernel_times(tm.h, reset=True)
@@ -327,6 +329,7 @@ def run_ours(args, rank, world, local_rank):
         L.llm_decode_step(tm.h, gen2[i], gen2[i + 1])
     kt_dec = L.llm_kernel_times(tm.h, reset=True)
     tm.free()
+    fused = kt_dec["step"][1] > 0  # decode steps ran as one launch each
     shares = {}
     for name, (ms, n) in kt_pre.items():
         if n:
@@ -366,11 +369,13 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": WORKLOAD, "batch": B, "prompt_len": T, "decode_steps": G,
                    "layers": shape.n_layers, "dim": shape.dim, "vocab": shape.vocab,
                    "l2": "inputs larger than L2: every step streams 16 GB of weights",
-                   "cuda_graph_decode": not args.no_graph, "parallelism": f"replicas x{world}"},
+                   "cuda_graph_decode": not args.no_graph, "decode_kernel": "fused step" if fused else "layerwise",
+                   "parallelism": f"replicas x{world}"},
         "prefill": prefill, "decode": decode, "roofline": roof, "kernels": kernel_table,
         "cpu_baseline": ({k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")} if cpu else None),
         "e2e": e2e,
-        "gpu_launches": args.steps * (G + 1) * (5 * shape.n_layers + 2),
+        "gpu_launches": args.steps * ((5 * shape.n_layers + 2) +
+                                      G * (1 if fused else 5 * shape.n_layers + 2)),
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
@@ -384,6 +389,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--layerwise", action="store_true",
+                    help="decode one launch per projection/attention instead of the fused step kernel")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -65,6 +65,10 @@ extern "C" {
 #define LLM_FLAG_PDL           8 /* let each kernel launch while the previous one drains
                                     (programmatic dependent launch); off by default because it
                                     unbalances the persistent one-CTA-per-SM projections */
+#define LLM_FLAG_LAYERWISE_DECODE 16 /* run bf16 decode steps as one launch per projection and
+                                    attention instead of the fused decode-step kernel (which
+                                    runs the whole step in one persistent launch); the fused
+                                    kernel is also skipped with LLM_FLAG_DEBUG_TAPS */
 
 /* ---- kernel kinds reported by llm_kernel_times ------------------------- */
 #define LLM_K_EMBED    0   /* embedding lookup / hidden-state load */
@@ -75,7 +79,8 @@ extern "C" {
 #define LLM_K_W2       5   /* w2 projection + residual */
 #define LLM_K_HEAD     6   /* final norm + lm_head + argmax */
 #define LLM_K_OUT      7   /* hidden-state output */
-#define LLM_K_COUNT    8
+#define LLM_K_STEP     8   /* fused decode step: the whole model in one launch */
+#define LLM_K_COUNT    9
 
 /*
  * Model hyper-parameters: the params.json fields of "Building llama3 from

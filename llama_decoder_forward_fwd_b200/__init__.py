@@ -30,7 +30,8 @@ LLM_FLAG_CUDA_GRAPH = 1
 LLM_FLAG_DEBUG_TAPS = 2
 LLM_FLAG_KERNEL_TIMING = 4
 LLM_FLAG_PDL = 8
-KERNEL_KINDS = ("embed", "qkv", "attn", "wo", "w13", "w2", "head", "out")
+LLM_FLAG_LAYERWISE_DECODE = 16
+KERNEL_KINDS = ("embed", "qkv", "attn", "wo", "w13", "w2", "head", "out", "step")
 
 
 class llm_config(ctypes.Structure):

@@ -91,7 +91,6 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 struct LayerW {
     const void *attn_norm, *wq, *wk, *wv, *wo, *ffn_norm, *w1, *w3, *w2;
 };
-enum { TM_WQ, TM_WK, TM_WV, TM_WO, TM_W1, TM_W3, TM_W2, TM_W1G, TM_W3G, TM_PER_LAYER };
 
 // RMSNorm partial sums written by a residual projection with N output rows.
 int bf16_gemv_ss_parts(int N) { return gemv_num_tiles(EPI_RESID, N) * 8; }  // one per 16 rows of a 128-row tile
@@ -139,6 +138,13 @@ struct llm_model {
     CUtensorMap tm_hw, tm_o, tm_g, tm_kc, tm_vc, tm_head;
     std::vector<CUtensorMap> tm_w;
     bool gemm_ok = false;
+    // fused decode step (bf16): device copies of the weight tensor maps and norm
+    // pointers, and the grid-barrier counter
+    bool fused = false;
+    int smem_optin = 0;
+    CUtensorMap* d_tmaps = nullptr;
+    const void** d_norms = nullptr;
+    unsigned* ds_bar = nullptr;
     // per-launch CUDA-event timing (LLM_FLAG_KERNEL_TIMING)
     bool timing = false;
     bool capturing = false;
@@ -522,8 +528,74 @@ int run_embed(llm_model* m, const int32_t* tok, const float* h_in, int M) {
     return LLM_OK;
 }
 
+DecodeStepPlan fused_plan(const llm_model* m, int B, int max_keys) {
+    const llm_config& c = m->cfg;
+    return decode_step_plan(B, c.dim, c.n_heads, c.n_kv_heads, c.head_dim, c.ffn_hidden, c.vocab,
+                            c.has_embed_and_head, max_keys, m->num_sms, m->smem_optin);
+}
+
+// One decode step of every sequence b < B as a single fused launch (token ids,
+// or hidden states for a bare layer stack).
+int run_fused_step(llm_model* m, int B, const int32_t* tok, const float* h_in, float* h_out, int32_t* next,
+                   float* logits) {
+    const llm_config& c = m->cfg;
+    const DecodeStepPlan p = fused_plan(m, B, max_keys_after(m, B, 1));
+    if (!p.supported) return fail(LLM_ERR_UNSUPPORTED, "fused decode step does not support this shape");
+    if (p.part_floats > m->gws.part_floats || p.tiles > m->gws.tiles_cap || p.attn_part_floats > m->attn_ws_floats ||
+        p.attn_counters > m->attn_cnt_n)
+        return fail(LLM_ERR_UNSUPPORTED, "fused decode step scratch too small for this call");
+    DecodeStepArgs a;
+    a.B = B;
+    a.D = c.dim;
+    a.H = c.n_heads;
+    a.Hk = c.n_kv_heads;
+    a.d = c.head_dim;
+    a.F = c.ffn_hidden;
+    a.vocab = c.vocab;
+    a.S_max = c.max_seq_len;
+    a.n_layers = c.n_layers;
+    a.eps = c.norm_eps;
+    a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)c.head_dim));
+    a.has_head = c.has_embed_and_head;
+    a.n_splits = p.n_splits;
+    a.n_stages = p.n_stages;
+    a.xs_bytes = p.xs_bytes;
+    for (int i = 0; i < 5; ++i) a.max_pieces[i] = p.max_pieces[i];
+    a.tok = tok;
+    a.h_in = h_in;
+    a.h_out = h_out;
+    a.next = next;
+    a.logits = logits;
+    a.tmaps = m->d_tmaps;
+    a.norms = m->d_norms;
+    a.tok_emb = m->tok_emb;
+    a.kc = m->kc;
+    a.vc = m->vc;
+    a.layer_elems = m->layer_elems;
+    a.seq_len = m->seq_len;
+    a.h = m->h;
+    a.hw = reinterpret_cast<__nv_bfloat16*>(m->hw);
+    a.ss = m->ss;
+    a.ss_ld = m->ss_ld;
+    a.q = reinterpret_cast<__nv_bfloat16*>(m->q);
+    a.o = reinterpret_cast<__nv_bfloat16*>(m->o);
+    a.g = reinterpret_cast<__nv_bfloat16*>(m->g);
+    a.rope_cos = m->rope_cos;
+    a.rope_sin = m->rope_sin;
+    a.ws = m->gws;
+    a.attn_part = m->attn_ws;
+    a.attn_cnt = m->attn_cnt;
+    a.bar = m->ds_bar;
+    a.err = m->d_err;
+    KTimer timer(m, LLM_K_STEP);
+    CK(cudaMemsetAsync(m->ds_bar, 0, 4, m->stream));
+    CK(launch_decode_step(a, p, m->stream));
+    return LLM_OK;
+}
+
 // The device work of one decode step (captured into a graph when enabled).
 int decode_core(llm_model* m, int B, const int32_t* tok, int32_t* next, float* logits) {
+    if (m->fused) return run_fused_step(m, B, tok, nullptr, nullptr, next, logits);
     int rc = run_embed(m, tok, nullptr, B);
     if (rc) return rc;
     rc = run_layers(m, B, 1, max_keys_after(m, B, 1));
@@ -725,6 +797,65 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
                 return bail(fail(LLM_ERR_CUDA, "cuTensorMapEncodeTiled (KV cache) failed"));
         }
     }
+    // Fused decode step: supported shapes only, sized for every batch size at the
+    // longest cache; its scratch is the decode projection's and the attention's.
+    if (m->bf16 && !(c.flags & (LLM_FLAG_LAYERWISE_DECODE | LLM_FLAG_DEBUG_TAPS))) {
+        cudaDeviceGetAttribute(&m->smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, m->dev);
+        int coop = 0;
+        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, m->dev);
+        bool ok = coop != 0;
+        size_t pf = 0, af = 0, ac = 0;
+        int tiles = 0;
+        for (int B = 1; B <= c.max_batch && ok; ++B) {
+            const DecodeStepPlan p = fused_plan(m, B, c.max_seq_len);
+            ok = p.supported;
+            pf = p.part_floats > pf ? p.part_floats : pf;
+            af = p.attn_part_floats > af ? p.attn_part_floats : af;
+            ac = p.attn_counters > ac ? p.attn_counters : ac;
+            tiles = p.tiles > tiles ? p.tiles : tiles;
+        }
+        if (ok) {
+            if (pf > m->gws.part_floats) {
+                MALLOC_OR_BAIL(m->gws.part, pf * 4);
+                m->gws.part_floats = pf;
+            }
+            if (tiles > m->gws.tiles_cap) {
+                MALLOC_OR_BAIL(m->gws.tile_cnt, (size_t)tiles * 4);
+                m->gws.tiles_cap = tiles;
+                if (cudaMemsetAsync(m->gws.tile_cnt, 0, (size_t)tiles * 4, m->stream) != cudaSuccess)
+                    return bail(fail(LLM_ERR_CUDA, "cudaMemsetAsync failed"));
+            }
+            if (af > m->attn_ws_floats) {
+                MALLOC_OR_BAIL(m->attn_ws, af * 4);
+                m->attn_ws_floats = af;
+            }
+            if (ac > m->attn_cnt_n) {
+                MALLOC_OR_BAIL(m->attn_cnt, ac * 4);
+                m->attn_cnt_n = ac;
+                if (cudaMemsetAsync(m->attn_cnt, 0, ac * 4, m->stream) != cudaSuccess)
+                    return bail(fail(LLM_ERR_CUDA, "cudaMemsetAsync failed"));
+            }
+            const size_t ntm = (size_t)c.n_layers * TM_PER_LAYER + 1;
+            std::vector<CUtensorMap> tms(m->tm_w);
+            tms.push_back(c.has_embed_and_head ? m->tm_head : m->tm_w[0]);
+            std::vector<const void*> norms;
+            for (int l = 0; l < c.n_layers; ++l) {
+                norms.push_back(m->L[l].attn_norm);
+                norms.push_back(m->L[l].ffn_norm);
+            }
+            norms.push_back(m->final_norm ? m->final_norm : m->L[c.n_layers - 1].ffn_norm);
+            MALLOC_OR_BAIL(m->d_tmaps, ntm * sizeof(CUtensorMap));
+            MALLOC_OR_BAIL(m->d_norms, norms.size() * sizeof(void*));
+            MALLOC_OR_BAIL(m->ds_bar, 64);
+            if (cudaMemcpyAsync(m->d_tmaps, tms.data(), ntm * sizeof(CUtensorMap), cudaMemcpyHostToDevice,
+                                m->stream) != cudaSuccess ||
+                cudaMemcpyAsync(m->d_norms, norms.data(), norms.size() * sizeof(void*), cudaMemcpyHostToDevice,
+                                m->stream) != cudaSuccess ||
+                cudaMemsetAsync(m->ds_bar, 0, 64, m->stream) != cudaSuccess)
+                return bail(fail(LLM_ERR_CUDA, "fused decode step setup copies failed"));
+            m->fused = true;
+        }
+    }
     if (cudaStreamSynchronize(m->stream) != cudaSuccess) return bail(fail(LLM_ERR_CUDA, "init sync failed"));
     *out = m;
     return LLM_OK;
@@ -769,9 +900,11 @@ int llm_decode_step(llm_model* m, int B, const int32_t* in_tok, int32_t* next, f
     if (rc) return rc;
     const size_t V = (size_t)m->cfg.vocab;
     if (m->cfg.flags & LLM_FLAG_CUDA_GRAPH) {
-        const AttnDecodePlan p = attn_decode_plan(B, 1, m->cfg.n_heads, m->cfg.n_kv_heads, m->cfg.head_dim,
-                                                  max_keys_after(m, B, 1), m->num_sms);
-        const auto key = std::make_tuple(B, p.n_splits, logits ? 1 : 0);
+        const int mk = max_keys_after(m, B, 1);
+        const int ns = m->fused ? fused_plan(m, B, mk).n_splits
+                                : attn_decode_plan(B, 1, m->cfg.n_heads, m->cfg.n_kv_heads, m->cfg.head_dim, mk,
+                                                   m->num_sms).n_splits;
+        const auto key = std::make_tuple(B, ns, logits ? 1 : 0);
         auto it = m->graphs.find(key);
         if (it == m->graphs.end()) {
             cudaGraph_t graph = nullptr;
@@ -816,7 +949,15 @@ int llm_decode_step(llm_model* m, int B, const int32_t* in_tok, int32_t* next, f
 }
 
 int llm_decode_step_hidden(llm_model* m, int B, const float* h_in, float* h_out) {
-    return llm_prefill_hidden(m, h_in, B, 1, h_out);
+    if (!m || !m->fused) return llm_prefill_hidden(m, h_in, B, 1, h_out);
+    if (!h_in || !h_out) return fail(LLM_ERR_NULL_PTR, "h_in or h_out is NULL");
+    if (!aligned16(h_in) || !aligned16(h_out)) return fail(LLM_ERR_BAD_ARG, "h_in and h_out must be 16-byte aligned");
+    int rc = check_batch(m, B, 1);
+    if (rc) return rc;
+    rc = run_fused_step(m, B, nullptr, h_in, h_out, nullptr, nullptr);
+    if (rc) return rc;
+    for (int b = 0; b < B; ++b) m->host_len[b] += 1;
+    return LLM_OK;
 }
 
 int llm_kv_cache_reset(llm_model* m) {

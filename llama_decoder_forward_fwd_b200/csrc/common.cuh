@@ -22,6 +22,9 @@ enum : uint32_t {
     DERR_ATTN_TMA_WAIT = 0x201,
     DERR_GEMV_PRODUCER_WAIT = 0x301,
     DERR_GEMV_CONSUMER_WAIT = 0x302,
+    DERR_GRID_BARRIER_WAIT = 0x401,
+    DERR_MK_PRODUCER_WAIT = 0x402,
+    DERR_MK_CONSUMER_WAIT = 0x403,
 };
 
 // 4 seconds: far longer than any legitimate wait for one pipeline stage.
@@ -83,6 +86,51 @@ DEVI bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err, uint32_t code
             return false;
         }
     }
+}
+
+DEVI unsigned ld_acquire_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Grid-wide barrier of a cooperative launch, entered by the first `nthreads`
+// threads of every CTA (the CTA's other warps do not take part). Barrier number
+// `index` (0, 1, 2, ...) of the launch waits until every CTA has arrived
+// `index + 1` times (*count is zero at launch). Writes made before the barrier
+// by any CTA are visible to every thread after it (release fence + arrival,
+// acquire polling, CTA barrier). The wait is bounded: on timeout it records
+// `code` in *err and returns false; it also returns false as soon as *err
+// holds another CTA's error, so all CTAs leave promptly.
+DEVI bool grid_barrier(unsigned* count, unsigned index, int nthreads, uint32_t* err, uint32_t code) {
+    __shared__ int gb_ok;
+    named_bar_sync(1, nthreads);
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(count, 1u);
+        const unsigned target = (index + 1) * gridDim.x;
+        int ok = 1;
+        if (ld_acquire_gpu(count) < target) {
+            const uint64_t t0 = globaltimer();
+            while (ld_acquire_gpu(count) < target) {
+                __nanosleep(32);
+                // leave at once if another CTA has already recorded an error
+                if (*reinterpret_cast<volatile uint32_t*>(err) != 0u) {
+                    ok = 0;
+                    break;
+                }
+                if (globaltimer() - t0 > kWaitLimitNs) {
+                    atomicCAS(err, 0u, code);
+                    ok = 0;
+                    break;
+                }
+            }
+        }
+        __threadfence();
+        gb_ok = ok;
+    }
+    named_bar_sync(1, nthreads);
+    return gb_ok != 0;
 }
 
 // ---- TMA --------------------------------------------------------------

@@ -107,7 +107,7 @@ DEVI float swiglu(float a, float c) { return silu(a) * c; }
 template <typename AT>
 DEVI float epi_resid1(const Epi& e, int m, int n, float v) {
     float* hp = e.h + (long long)m * e.D + n;
-    const float hn = *hp + v;
+    const float hn = __ldcg(hp) + v;  // h may have been written by another CTA earlier in this launch
     *hp = hn;
     const float w = to_f<AT>(reinterpret_cast<const AT*>(e.wnext)[n]);
     reinterpret_cast<AT*>(e.hw_out)[(long long)m * e.D + n] = from_f<AT>(hn * w);

@@ -75,6 +75,11 @@ struct Epi {
     uint32_t* err = nullptr;
 };
 
+// Tensor maps of one layer's weights, in this order per layer: 128-row boxes
+// for the decode projection and the prefill GEMM, and 64-row boxes of w1 and
+// w3 for the SwiGLU tiles of the decode projection.
+enum { TM_WQ, TM_WK, TM_WV, TM_WO, TM_W1, TM_W3, TM_W2, TM_W1G, TM_W3G, TM_PER_LAYER };
+
 // ---- decode projection: y = x W^T for M <= 16 token rows ---------------
 // Device scratch of the streaming bf16 GEMV. Counters and packed maxima must be
 // zero before the first launch; every launch leaves them zero again.
@@ -164,6 +169,57 @@ struct AttnDecodePlan {
 AttnDecodePlan attn_decode_plan(int B, int T, int H, int Hk, int d, int max_keys, int num_sms);
 cudaError_t launch_attn_decode(const AttnDecodeArgs& a, bool bf16, cudaStream_t s, bool pdl);
 cudaError_t attn_decode_prepare();
+
+// ---- fused decode step (bf16): the whole model in one persistent launch ----
+struct DecodeStepArgs {
+    int B = 0, D = 0, H = 0, Hk = 0, d = 0, F = 0, vocab = 0, S_max = 0, n_layers = 0;
+    float eps = 0.f, scale_log2 = 0.f;
+    int has_head = 0;
+    int n_splits = 1;                // attention key splits
+    int n_stages = 0, xs_bytes = 0;  // shared memory: ring stages; token rows / attention scratch
+    int max_pieces[5] = {1, 1, 1, 1, 1};  // split-tile slots of QKV, wo, w1/w3, w2, lm_head
+    // inputs and outputs of the step
+    const int32_t* tok = nullptr;  // [B] token ids (models with embedding and head)
+    const float* h_in = nullptr;   // [B][D] hidden states (layer stack only)
+    float* h_out = nullptr;        // [B][D]
+    int32_t* next = nullptr;       // [B] greedy next tokens
+    float* logits = nullptr;       // [B][vocab] or nullptr
+    // weights
+    const CUtensorMap* tmaps = nullptr;  // device: TM_PER_LAYER maps per layer, then the lm_head map
+    const void* const* norms = nullptr;  // device: attention_norm[l], ffn_norm[l] per layer, then the final norm
+    const void* tok_emb = nullptr;
+    // state and activations (layouts as above)
+    void* kc = nullptr;
+    void* vc = nullptr;
+    long long layer_elems = 0;
+    int32_t* seq_len = nullptr;
+    float* h = nullptr;
+    __nv_bfloat16* hw = nullptr;
+    float* ss = nullptr;
+    int ss_ld = 0;
+    __nv_bfloat16* q = nullptr;
+    __nv_bfloat16* o = nullptr;
+    __nv_bfloat16* g = nullptr;
+    const float* rope_cos = nullptr;
+    const float* rope_sin = nullptr;
+    // scratch (counters zero between launches; *bar zeroed before each launch)
+    GemvScratch ws;
+    float* attn_part = nullptr;
+    unsigned* attn_cnt = nullptr;
+    unsigned* bar = nullptr;
+    uint32_t* err = nullptr;
+};
+struct DecodeStepPlan {
+    bool supported;
+    int grid, rmax, n_splits, n_stages, xs_bytes, smem;
+    int max_pieces[5];
+    size_t part_floats;  // split-tile partial floats needed
+    int tiles;           // tile counters needed
+    size_t attn_part_floats, attn_counters;
+};
+DecodeStepPlan decode_step_plan(int B, int D, int H, int Hk, int d, int F, int vocab, int has_head, int max_keys,
+                                int num_sms, int smem_optin);
+cudaError_t launch_decode_step(const DecodeStepArgs& a, const DecodeStepPlan& p, cudaStream_t s);
 
 // ---- small kernels ----------------------------------------------------
 struct EmbedArgs {

@@ -19,10 +19,13 @@ def rel_l2(a, b) -> float:
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
 
 
-def build_pair(shape, seed, batch, max_tokens=0, flags=0):
+def build_pair(shape, seed, batch, max_tokens=0, flags=0, taps=True):
+    """GPU model and oracle on the same weights. With taps the GPU model keeps every
+    layer's output (which runs decode steps layer by layer); without, bf16 decode
+    steps run as the fused single-launch kernel."""
     glob, layers = S.make_weights(shape, seed)
     model = L.Model(shape, glob, layers, max_batch=batch, max_tokens=max_tokens,
-                    flags=flags | L.LLM_FLAG_DEBUG_TAPS)
+                    flags=flags | (L.LLM_FLAG_DEBUG_TAPS if taps else 0))
     orc = O.OracleModel(shape, glob, layers, batch)
     return model, orc
 
