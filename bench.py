@@ -199,15 +199,18 @@ def run_reference(args, rank):
 
 # ---------------------------------------------------------------- ncu traffic record
 def ncu_traffic(kind):
-    """DRAM bytes per launch of a kernel kind from the committed ncu summary, if it is current."""
+    """DRAM bytes per launch of a kernel kind from the committed ncu summary, if its
+    sources are unchanged since the counters were taken (else None)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
     rec = json.load(open(path)).get(kind)
     if not rec:
         return None
-    src = open(os.path.join(ROOT, "llama_decoder_forward_fwd_b200", "csrc", rec["source"]), "rb").read()
-    if hashlib.sha256(src).hexdigest()[:16] != rec["source_sha"]:
+    h = hashlib.sha256()
+    for f in rec["sources"]:
+        h.update(open(os.path.join(ROOT, "llama_decoder_forward_fwd_b200", "csrc", f), "rb").read())
+    if h.hexdigest()[:16] != rec["source_sha"]:
         return None  # the kernel changed since the counters were taken
     return rec["dram_bytes_per_launch"]
 
@@ -232,7 +235,7 @@ def run_ours(args, rank, world, local_rank):
 
     glob, layers = S.make_weights(shape, w.seed, device=dev)
     stream = torch.cuda.Stream(device=dev)
-    extra = L.LLM_FLAG_LAYERWISE_DECODE if args.layerwise else 0
+    extra = L.LLM_FLAG_FUSED_DECODE if args.fused else 0
     model = L.Model(shape, glob, layers, max_batch=B, max_tokens=B * T,
                     flags=extra | (0 if args.no_graph else L.LLM_FLAG_CUDA_GRAPH), stream=stream, device=dev)
     prompt = S.make_tokens(w.seed, B, T, shape.vocab).to(dev)
@@ -389,8 +392,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
-    ap.add_argument("--layerwise", action="store_true",
-                    help="decode one launch per projection/attention instead of the fused step kernel")
+    ap.add_argument("--fused", action="store_true",
+                    help="decode each step as the fused single-launch kernel instead of one launch per "
+                         "projection and attention")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -65,10 +65,12 @@ extern "C" {
 #define LLM_FLAG_PDL           8 /* let each kernel launch while the previous one drains
                                     (programmatic dependent launch); off by default because it
                                     unbalances the persistent one-CTA-per-SM projections */
-#define LLM_FLAG_LAYERWISE_DECODE 16 /* run bf16 decode steps as one launch per projection and
-                                    attention instead of the fused decode-step kernel (which
-                                    runs the whole step in one persistent launch); the fused
-                                    kernel is also skipped with LLM_FLAG_DEBUG_TAPS */
+#define LLM_FLAG_FUSED_DECODE  16 /* run each bf16 decode step as one persistent launch (the
+                                    whole model: every layer's projections and attention and the
+                                    lm_head, separated by grid barriers) instead of one launch per
+                                    projection and attention; needs head_dim 128 and a dim that
+                                    is a multiple of 256, and is not used with
+                                    LLM_FLAG_DEBUG_TAPS */
 
 /* ---- kernel kinds reported by llm_kernel_times ------------------------- */
 #define LLM_K_EMBED    0   /* embedding lookup / hidden-state load */

@@ -30,7 +30,7 @@ LLM_FLAG_CUDA_GRAPH = 1
 LLM_FLAG_DEBUG_TAPS = 2
 LLM_FLAG_KERNEL_TIMING = 4
 LLM_FLAG_PDL = 8
-LLM_FLAG_LAYERWISE_DECODE = 16
+LLM_FLAG_FUSED_DECODE = 16
 KERNEL_KINDS = ("embed", "qkv", "attn", "wo", "w13", "w2", "head", "out", "step")
 
 

@@ -20,6 +20,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <map>
@@ -142,6 +143,8 @@ struct llm_model {
     // pointers, and the grid-barrier counter
     bool fused = false;
     int smem_optin = 0;
+    int fused_prefetch = 0;  // L2 prefetch distance of the fused step (LLM_FUSED_PREFETCH_UNITS)
+    int fused_inflight = 0;  // weight copies in flight per SM (LLM_FUSED_INFLIGHT_UNITS)
     CUtensorMap* d_tmaps = nullptr;
     const void** d_norms = nullptr;
     unsigned* ds_bar = nullptr;
@@ -557,9 +560,10 @@ int run_fused_step(llm_model* m, int B, const int32_t* tok, const float* h_in, f
     a.eps = c.norm_eps;
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)c.head_dim));
     a.has_head = c.has_embed_and_head;
-    a.n_splits = p.n_splits;
     a.n_stages = p.n_stages;
     a.xs_bytes = p.xs_bytes;
+    a.prefetch_units = m->fused_prefetch;
+    a.inflight_units = m->fused_inflight;
     for (int i = 0; i < 5; ++i) a.max_pieces[i] = p.max_pieces[i];
     a.tok = tok;
     a.h_in = h_in;
@@ -572,6 +576,7 @@ int run_fused_step(llm_model* m, int B, const int32_t* tok, const float* h_in, f
     a.kc = m->kc;
     a.vc = m->vc;
     a.layer_elems = m->layer_elems;
+    a.kv_rows_per_layer = m->layer_elems / c.head_dim;
     a.seq_len = m->seq_len;
     a.h = m->h;
     a.hw = reinterpret_cast<__nv_bfloat16*>(m->hw);
@@ -745,6 +750,7 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
         MALLOC_OR_BAIL(m->gws.tile_cnt, (size_t)tiles * 4);
         MALLOC_OR_BAIL(m->gws.am_best, 16 * 8);
         MALLOC_OR_BAIL(m->gws.done_cnt, 16);
+        MALLOC_OR_BAIL(m->gws.warp_cnt, (size_t)tiles * 8 * 4);
     }
     MALLOC_OR_BAIL(m->d_tok, (size_t)c.max_batch * 4);
     MALLOC_OR_BAIL(m->d_next, (size_t)c.max_batch * 4);
@@ -760,7 +766,8 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
         cudaMemsetAsync(m->ss, 0, (size_t)parts * Mx * 4, m->stream) != cudaSuccess ||
         (m->bf16 && (cudaMemsetAsync(m->gws.tile_cnt, 0, (size_t)m->gws.tiles_cap * 4, m->stream) != cudaSuccess ||
                      cudaMemsetAsync(m->gws.am_best, 0, 16 * 8, m->stream) != cudaSuccess ||
-                     cudaMemsetAsync(m->gws.done_cnt, 0, 16, m->stream) != cudaSuccess)))
+                     cudaMemsetAsync(m->gws.done_cnt, 0, 16, m->stream) != cudaSuccess ||
+                     cudaMemsetAsync(m->gws.warp_cnt, 0, (size_t)m->gws.tiles_cap * 8 * 4, m->stream) != cudaSuccess)))
         return bail(fail(LLM_ERR_CUDA, "cudaMemsetAsync failed"));
     if (attn_decode_prepare() != cudaSuccess) return bail(fail(LLM_ERR_CUDA, "attention kernel attributes"));
     if (launch_rope_tables(m->rope_cos, m->rope_sin, c.max_seq_len, d / 2, (double)c.rope_theta, d, m->stream) !=
@@ -799,7 +806,7 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
     }
     // Fused decode step: supported shapes only, sized for every batch size at the
     // longest cache; its scratch is the decode projection's and the attention's.
-    if (m->bf16 && !(c.flags & (LLM_FLAG_LAYERWISE_DECODE | LLM_FLAG_DEBUG_TAPS))) {
+    if (m->bf16 && (c.flags & LLM_FLAG_FUSED_DECODE) && !(c.flags & LLM_FLAG_DEBUG_TAPS)) {
         cudaDeviceGetAttribute(&m->smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, m->dev);
         int coop = 0;
         cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, m->dev);
@@ -821,8 +828,10 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
             }
             if (tiles > m->gws.tiles_cap) {
                 MALLOC_OR_BAIL(m->gws.tile_cnt, (size_t)tiles * 4);
+                MALLOC_OR_BAIL(m->gws.warp_cnt, (size_t)tiles * 8 * 4);
                 m->gws.tiles_cap = tiles;
-                if (cudaMemsetAsync(m->gws.tile_cnt, 0, (size_t)tiles * 4, m->stream) != cudaSuccess)
+                if (cudaMemsetAsync(m->gws.tile_cnt, 0, (size_t)tiles * 4, m->stream) != cudaSuccess ||
+                    cudaMemsetAsync(m->gws.warp_cnt, 0, (size_t)tiles * 8 * 4, m->stream) != cudaSuccess)
                     return bail(fail(LLM_ERR_CUDA, "cudaMemsetAsync failed"));
             }
             if (af > m->attn_ws_floats) {
@@ -835,9 +844,18 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
                 if (cudaMemsetAsync(m->attn_cnt, 0, ac * 4, m->stream) != cudaSuccess)
                     return bail(fail(LLM_ERR_CUDA, "cudaMemsetAsync failed"));
             }
-            const size_t ntm = (size_t)c.n_layers * TM_PER_LAYER + 1;
+            const size_t ntm = (size_t)c.n_layers * TM_PER_LAYER + 3;
             std::vector<CUtensorMap> tms(m->tm_w);
             tms.push_back(c.has_embed_and_head ? m->tm_head : m->tm_w[0]);
+            {
+                // the whole K and V caches as [rows][head_dim], 32-row boxes (attention units)
+                const uint64_t rows = (uint64_t)c.n_layers * c.max_batch * Hk * c.max_seq_len;
+                CUtensorMap k32, v32;
+                if (!make_tmap(&k32, m->kc, d, rows, 64, 32) || !make_tmap(&v32, m->vc, d, rows, 64, 32))
+                    return bail(fail(LLM_ERR_CUDA, "cuTensorMapEncodeTiled (KV cache, fused step) failed"));
+                tms.push_back(k32);
+                tms.push_back(v32);
+            }
             std::vector<const void*> norms;
             for (int l = 0; l < c.n_layers; ++l) {
                 norms.push_back(m->L[l].attn_norm);
@@ -854,6 +872,10 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
                 cudaMemsetAsync(m->ds_bar, 0, 64, m->stream) != cudaSuccess)
                 return bail(fail(LLM_ERR_CUDA, "fused decode step setup copies failed"));
             m->fused = true;
+            if (const char* pe = getenv("LLM_FUSED_PREFETCH_UNITS")) m->fused_prefetch = atoi(pe);
+            if (m->fused_prefetch < 0) m->fused_prefetch = 0;
+            if (const char* ie = getenv("LLM_FUSED_INFLIGHT_UNITS")) m->fused_inflight = atoi(ie);
+            if (m->fused_inflight < 0) m->fused_inflight = 0;
         }
     }
     if (cudaStreamSynchronize(m->stream) != cudaSuccess) return bail(fail(LLM_ERR_CUDA, "init sync failed"));
@@ -901,7 +923,8 @@ int llm_decode_step(llm_model* m, int B, const int32_t* in_tok, int32_t* next, f
     const size_t V = (size_t)m->cfg.vocab;
     if (m->cfg.flags & LLM_FLAG_CUDA_GRAPH) {
         const int mk = max_keys_after(m, B, 1);
-        const int ns = m->fused ? fused_plan(m, B, mk).n_splits
+        // the fused step splits the attention at run time from the cache lengths
+        const int ns = m->fused ? 0
                                 : attn_decode_plan(B, 1, m->cfg.n_heads, m->cfg.n_kv_heads, m->cfg.head_dim, mk,
                                                    m->num_sms).n_splits;
         const auto key = std::make_tuple(B, ns, logits ? 1 : 0);

@@ -148,6 +148,13 @@ DEVI void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int
         : "memory");
 }
 
+// Prefetch of the same 2-D box into L2 only (no shared memory, no completion).
+DEVI void tma_prefetch_l2_2d(const CUtensorMap* m, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(m)),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
+
 // Untiled bulk copy global -> shared (both 16-byte aligned, bytes % 16 == 0).
 DEVI void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
     asm volatile(

@@ -19,10 +19,20 @@
 //
 // Phase order per layer: QKV -> attention -> wo -> w1/w3 -> w2, each ending in a
 // grid barrier (the data dependency is all-to-all: every projection row needs
-// the whole input vector). The arithmetic of each phase is the same code as the
-// per-projection kernels (gemv_core.cuh, attn_core.cuh), so results agree with
-// the layer-by-layer path up to the split of the k sums over CTAs (which is a
-// function of the grid size only, so a given GPU gives bit-identical steps).
+// the whole input vector). The projections are the code of the per-projection
+// kernel (gemv_core.cuh), except that a split row tile is finished by its first
+// CTA. The attention phase streams the KV cache through the same ring: a unit
+// is the K and V tiles of 32 keys of one (sequence, KV head) group, and the
+// units of all groups are split evenly over the CTAs. Each consumer warp owns
+// 16 of the 128 output dims: it computes S = Q K^T for the group's query heads
+// (padded to 16 rows) with mma.sync from the swizzled tiles, keeps the online
+// softmax (running max and sum, log2 domain) and accumulates P V for its dims.
+// A group split over several CTAs is merged by its first CTA (log-sum-exp
+// rule, pieces in CTA order). The ring may have fetched the tile that holds the
+// new token before this step's QKV phase wrote its key and value, so the CTA
+// that owns that tile patches the row from the cache before using it.
+// Reductions are split by a function of the grid size and the cache lengths
+// only, so a given GPU gives bit-identical steps.
 //
 // Barrier waits, ring waits and the final drain are all bounded; a timeout
 // records an error code and every CTA leaves at its next barrier.
@@ -98,7 +108,319 @@ DEVI void ds_embed(const DecodeStepArgs& a) {
 
 // 9 warps per CTA put 3 warps on one of the SM's four register partitions
 // (16K registers each), so a thread gets at most 168 registers.
-template <int NB, int RMAX>
+constexpr int AK = 32;  // keys per attention unit (K and V tiles of 32 x 128 bf16 = 16 KB)
+
+// Swizzled address of 16-byte chunk `chunk` (0..15) of key row `key` in a K or V
+// tile of an attention unit: two 64-dim halves of 32 rows x 128 B, 4 KB apart.
+DEVI uint32_t kv32_addr(uint32_t base, int key, int chunk) {
+    return base + (chunk >> 3) * (AK * 128) + key * 128 + (((chunk & 7) ^ (key & 7)) << 4);
+}
+// Attention units of a group: keys 0 .. len (the new token at position len).
+DEVI int group_units(const int* s_len, int grp, int Hk) { return (s_len[grp / Hk] + AK) / AK; }
+
+// This CTA's share of the attention units (the same for every layer).
+struct AttnSplit {
+    long long U, G, u0, u1;  // all units, CTAs taking part, this CTA's range
+    int g0, j0;              // group and tile of unit u0
+    long long cum0;          // first unit of group g0
+};
+DEVI AttnSplit attn_split(const int* s_len, int B, int Hk) {
+    AttnSplit sp;
+    long long U = 0;
+    for (int gr = 0; gr < B * Hk; ++gr) U += group_units(s_len, gr, Hk);
+    sp.U = U;
+    sp.G = (long long)gridDim.x < U ? (long long)gridDim.x : U;
+    if (blockIdx.x < sp.G) {
+        sp.u0 = blockIdx.x * U / sp.G;
+        sp.u1 = (blockIdx.x + 1) * U / sp.G;
+    } else {
+        sp.u0 = sp.u1 = U;
+    }
+    long long c = 0;
+    int gr = 0;
+    while (gr < B * Hk) {
+        const int n = group_units(s_len, gr, Hk);
+        if (c + n > sp.u0) break;
+        c += n;
+        ++gr;
+    }
+    sp.g0 = gr;
+    sp.j0 = (int)(sp.u0 - c);
+    sp.cum0 = c;
+    return sp;
+}
+
+// Producer: the TMA copies of this CTA's attention units of layer l (K and V
+// tiles of 32 keys, each as two 64-dim boxes).
+DEVI bool attn_produce(GvRing& r, const DecodeStepArgs& a, int l, const AttnSplit& sp, const int* s_len) {
+    const CUtensorMap* tk = a.tmaps + (size_t)a.n_layers * TM_PER_LAYER + 1;
+    const CUtensorMap* tv = tk + 1;
+    int gr = sp.g0, j = sp.j0;
+    int n = sp.u0 < sp.u1 ? group_units(s_len, gr, a.Hk) : 0;
+    for (long long u = sp.u0; u < sp.u1; ++u) {
+        if (!mbar_wait(&r.empty[r.st], r.ph ^ 1u, a.err, DERR_MK_PRODUCER_WAIT)) return false;
+        if (!ring_throttle(r, a.err, DERR_MK_PRODUCER_WAIT)) return false;
+        uint8_t* dst = r.stages + r.st * GV_UNIT_BYTES;
+        const int row = (int)((long long)l * a.kv_rows_per_layer + (long long)gr * a.S_max + j * AK);
+        mbar_arrive_expect_tx(&r.full[r.st], GV_UNIT_BYTES);
+        tma_load_2d(dst, tk, &r.full[r.st], 0, row);
+        tma_load_2d(dst + AK * 128, tk, &r.full[r.st], 64, row);
+        tma_load_2d(dst + 2 * AK * 128, tv, &r.full[r.st], 0, row);
+        tma_load_2d(dst + 3 * AK * 128, tv, &r.full[r.st], 64, row);
+        if (++j == n) {
+            j = 0;
+            ++gr;
+            if (u + 1 < sp.u1) n = group_units(s_len, gr, a.Hk);
+        }
+        ++r.issued;
+        ring_next(r);
+    }
+    return true;
+}
+
+// Consumers: this CTA's attention units of layer l (see the file comment).
+// qsm: 4 KB of 1024-aligned shared memory for the group's query rows.
+DEVI void attn_consume(GvRing& ring, const DecodeStepArgs& a, int l, const AttnSplit& sp, const int* s_len,
+                       uint8_t* qsm) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g8 = lane >> 2, t4 = lane & 3, j8 = lane >> 3, i8 = lane & 7;
+    const int Hk = a.Hk, R = a.H / a.Hk, HD = a.H * 128;
+    const __nv_bfloat16* kc = reinterpret_cast<const __nv_bfloat16*>(a.kc) + (size_t)l * a.layer_elems;
+    const __nv_bfloat16* vc = reinterpret_cast<const __nv_bfloat16*>(a.vc) + (size_t)l * a.layer_elems;
+    const uint32_t qbase = smem_u32(qsm);
+    const long long G = sp.G;
+    bool ok = true;
+    int gr = sp.g0, jt = sp.j0, n_g = 0, p0 = 0;
+    long long cum = sp.cum0;
+    bool fresh = true;
+    uint32_t qf[8][4];
+    float o[2][4], mrow[2], lrow[2];
+    uint4 patch = make_uint4(0, 0, 0, 0);
+
+    // Publishes this CTA's piece of group gr, or (first CTA of the group) merges
+    // all pieces, and writes the group's attention output rows.
+    auto finish_group = [&]() {
+        const int b = gr / Hk, kvh = gr % Hk;
+        const long long cf = cta_of_unit(cum, G, sp.U), cl = cta_of_unit(cum + n_g - 1, G, sp.U);
+        const long long pc = blockIdx.x - cf;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            lrow[hh] += __shfl_xor_sync(0xffffffffu, lrow[hh], 1);
+            lrow[hh] += __shfl_xor_sync(0xffffffffu, lrow[hh], 2);
+        }
+        const size_t rec_floats = 18 * (size_t)R;  // per warp: O[R][16], m[R], l[R]
+        float* recs = a.attn_part + (size_t)gr * gridDim.x * 8 * rec_floats;
+        unsigned* cnt = a.attn_cnt + gr * 8 + warp;
+        if (cf != cl && pc != 0) {
+            float* rec = recs + ((size_t)pc * 8 + warp) * rec_floats;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int row = g8 + 8 * hh;
+                if (row >= R) continue;
+#pragma unroll
+                for (int n = 0; n < 2; ++n)
+                    *reinterpret_cast<float2*>(rec + row * 16 + n * 8 + 2 * t4) = make_float2(o[n][2 * hh], o[n][2 * hh + 1]);
+                if (t4 == 0) {
+                    rec[16 * R + row] = mrow[hh];
+                    rec[17 * R + row] = lrow[hh];
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence();
+                atomicAdd(cnt, 1u);
+            }
+            __syncwarp();
+            return;
+        }
+        if (cf != cl) {
+            if (lane == 0) {
+                const unsigned want = (unsigned)(cl - cf);
+                if (ld_acquire_gpu(cnt) < want) {
+                    const uint64_t t0 = globaltimer();
+                    while (ld_acquire_gpu(cnt) < want) {
+                        if (globaltimer() - t0 > kWaitLimitNs) {
+                            atomicCAS(a.err, 0u, DERR_MK_CONSUMER_WAIT);
+                            break;
+                        }
+                    }
+                }
+                *cnt = 0u;
+            }
+            __syncwarp();
+            // log-sum-exp merge of the pieces, in CTA order; the loads of PB pieces
+            // are issued together
+            constexpr int PB = 2;
+            const int np = (int)(cl - cf);
+            for (int p0 = 1; p0 <= np; p0 += PB) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int row = g8 + 8 * hh;
+                    if (row >= R) continue;
+                    float mp[PB], lp[PB];
+                    float2 o0[PB], o1[PB];
+#pragma unroll
+                    for (int q = 0; q < PB; ++q) {
+                        if (p0 + q > np) continue;
+                        const float* rec = recs + ((size_t)(p0 + q) * 8 + warp) * rec_floats;
+                        mp[q] = __ldcg(rec + 16 * R + row);
+                        lp[q] = __ldcg(rec + 17 * R + row);
+                        o0[q] = __ldcg(reinterpret_cast<const float2*>(rec + row * 16 + 2 * t4));
+                        o1[q] = __ldcg(reinterpret_cast<const float2*>(rec + row * 16 + 8 + 2 * t4));
+                    }
+#pragma unroll
+                    for (int q = 0; q < PB; ++q) {
+                        if (p0 + q > np) continue;
+                        const float mn = fmaxf(mrow[hh], mp[q]);
+                        const float mu = mn == -INFINITY ? 0.f : mn;
+                        const float sa = exp2f(mrow[hh] - mu), sb = exp2f(mp[q] - mu);
+                        lrow[hh] = lrow[hh] * sa + lp[q] * sb;
+                        o[0][2 * hh] = o[0][2 * hh] * sa + o0[q].x * sb;
+                        o[0][2 * hh + 1] = o[0][2 * hh + 1] * sa + o0[q].y * sb;
+                        o[1][2 * hh] = o[1][2 * hh] * sa + o1[q].x * sb;
+                        o[1][2 * hh + 1] = o[1][2 * hh + 1] * sa + o1[q].y * sb;
+                        mrow[hh] = mn;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int row = g8 + 8 * hh;
+            if (row >= R) continue;
+            const float inv = lrow[hh] > 0.f ? 1.f / lrow[hh] : 0.f;
+            __nv_bfloat16* dst = a.o + (size_t)b * HD + (kvh * R + row) * 128 + 16 * warp + 2 * t4;
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+                *reinterpret_cast<uint32_t*>(dst + n * 8) = pack_bf16x2(o[n][2 * hh] * inv, o[n][2 * hh + 1] * inv);
+        }
+    };
+
+    for (long long u = sp.u0; u < sp.u1; ++u) {
+        if (fresh) {
+            // entering group gr: its query rows (zero past R), and the new token's
+            // key and value row if this CTA holds the group's last tile
+            const int b = gr / Hk, kvh = gr % Hk;
+            n_g = group_units(s_len, gr, Hk);
+            p0 = s_len[b];
+            named_bar_sync(1, GV_CONSUMERS);  // the previous group's query rows are no longer read
+            if (warp == 0 && cum + n_g - 1 < sp.u1) {
+                const __nv_bfloat16* src = (lane < 16 ? kc : vc) + ((size_t)gr * a.S_max + p0) * 128 + (lane & 15) * 8;
+                patch = __ldcg(reinterpret_cast<const uint4*>(src));
+            }
+            {
+                const int r = threadIdx.x >> 4, c = threadIdx.x & 15;
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (r < R) v = __ldcg(reinterpret_cast<const uint4*>(a.q + (size_t)b * HD + (kvh * R + r) * 128 + c * 8));
+                *reinterpret_cast<uint4*>(qsm + r * 256 + ((c ^ (r & 7)) << 4)) = v;
+            }
+            named_bar_sync(1, GV_CONSUMERS);
+            {
+                const int r = (j8 & 1) * 8 + i8;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const int c = 2 * kk + (j8 >> 1);
+                    ldsm_x4(qf[kk], qbase + r * 256 + ((c ^ (r & 7)) << 4));
+                }
+            }
+#pragma unroll
+            for (int n = 0; n < 2; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+            mrow[0] = mrow[1] = -INFINITY;
+            lrow[0] = lrow[1] = 0.f;
+            fresh = false;
+        }
+        if (ok && !mbar_wait(&ring.full[ring.st], ring.ph, a.err, DERR_MK_CONSUMER_WAIT)) ok = false;
+        const uint32_t kb = smem_u32(ring.stages + ring.st * GV_UNIT_BYTES);
+        const uint32_t vb = kb + 2 * AK * 128;
+        const int key0 = jt * AK;
+        if (key0 <= p0 && p0 < key0 + AK) {
+            // the new token's row, written by this step's QKV phase
+            if (warp == 0) {
+                const uint32_t dst = kv32_addr(lane < 16 ? kb : vb, p0 - key0, lane & 15);
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(patch.x), "r"(patch.y), "r"(patch.z),
+                             "r"(patch.w)
+                             : "memory");
+                fence_proxy_async();  // before the stage is handed back to the TMA writes
+            }
+            named_bar_sync(1, GV_CONSUMERS);
+        }
+        // S = Q K^T: 16 (padded) query rows x 32 keys
+        float sc[4][4];
+#pragma unroll
+        for (int n = 0; n < 4; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t rr[4];
+                ldsm_x4(rr, kv32_addr(kb, (2 * np + (j8 >> 1)) * 8 + i8, 2 * kk + (j8 & 1)));
+                mma_bf16_16816(sc[2 * np], qf[kk], rr[0], rr[1]);
+                mma_bf16_16816(sc[2 * np + 1], qf[kk], rr[2], rr[3]);
+            }
+        }
+        // online softmax over the unit's keys (keys after the new token masked)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int n = 0; n < 4; ++n)
+#pragma unroll
+                for (int e2 = 0; e2 < 2; ++e2) {
+                    float v = sc[n][2 * hh + e2] * a.scale_log2;
+                    if (key0 + n * 8 + 2 * t4 + e2 > p0) v = -INFINITY;
+                    sc[n][2 * hh + e2] = v;
+                    mx = fmaxf(mx, v);
+                }
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float mnew = fmaxf(mrow[hh], mx);
+            const float muse = mnew == -INFINITY ? 0.f : mnew;
+            const float alpha = exp2f(mrow[hh] - muse);
+            mrow[hh] = mnew;
+            float sum = 0.f;
+#pragma unroll
+            for (int n = 0; n < 4; ++n)
+#pragma unroll
+                for (int e2 = 0; e2 < 2; ++e2) {
+                    const float pv = exp2f(sc[n][2 * hh + e2] - muse);
+                    sc[n][2 * hh + e2] = pv;
+                    sum += pv;
+                }
+            lrow[hh] = lrow[hh] * alpha + sum;
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+                o[n][2 * hh] *= alpha;
+                o[n][2 * hh + 1] *= alpha;
+            }
+        }
+        // O += P V for this warp's 16 dims
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            uint32_t pf[4];
+            pf[0] = pack_bf16x2(sc[2 * ks][0], sc[2 * ks][1]);
+            pf[1] = pack_bf16x2(sc[2 * ks][2], sc[2 * ks][3]);
+            pf[2] = pack_bf16x2(sc[2 * ks + 1][0], sc[2 * ks + 1][1]);
+            pf[3] = pack_bf16x2(sc[2 * ks + 1][2], sc[2 * ks + 1][3]);
+            uint32_t rr[4];
+            ldsm_x4_t(rr, kv32_addr(vb, ks * 16 + (j8 & 1) * 8 + i8, 2 * warp + (j8 >> 1)));
+            mma_bf16_16816(o[0], pf, rr[0], rr[1]);
+            mma_bf16_16816(o[1], pf, rr[2], rr[3]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ring.empty[ring.st]);
+        ring_next(ring);
+        if (++jt == n_g) {
+            finish_group();
+            cum += n_g;
+            ++gr;
+            jt = 0;
+            fresh = true;
+        }
+    }
+    if (!fresh) finish_group();
+}
+
+template <int NB>
 __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const DecodeStepArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -107,7 +429,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
     __shared__ float rinv_s[16];
     __shared__ float rred_s[8][16];
     __shared__ int last_s;
-    GvRing ring{smem, full, full + a.n_stages, a.n_stages, 0, 0u};
+    __shared__ int s_len[16];  // cache lengths before this step (the new token's positions)
+    GvRing ring{smem, full, full + a.n_stages, a.n_stages, 0, 0u, a.inflight_units, 0};
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const int B = a.B, D = a.D, Hd = a.H * a.d, Hkd = a.Hk * a.d, F = a.F;
@@ -122,10 +445,12 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
         }
         fence_mbar_init();
     }
+    if (threadIdx.x < B) s_len[threadIdx.x] = a.seq_len[threadIdx.x];
     __syncthreads();
+    const AttnSplit asp = attn_split(s_len, B, a.Hk);
 
     if (warp == DS_NW) {
-        // ---------------- producer: every phase's weight units, back to back ----------------
+        // ---------------- producer: every phase's units, back to back ----------------
         if (lane == 0) {
             bool ok = true;
             long long issued = 0;
@@ -134,6 +459,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
                 GvWork w = gv_work(nt_qkv, nku_D);
                 ok = ok && gv_produce(ring, w, false, t + TM_WQ, t + TM_WK, t + TM_WV, Hd, Hkd, a.err, DERR_MK_PRODUCER_WAIT);
                 issued += w.u1 - w.u0;
+                ok = ok && attn_produce(ring, a, l, asp, s_len);
+                issued += asp.u1 - asp.u0;
                 w = gv_work(nt_D, nku_Hd);
                 ok = ok && gv_produce(ring, w, false, t + TM_WO, t + TM_WO, t + TM_WO, 0, 0, a.err, DERR_MK_PRODUCER_WAIT);
                 issued += w.u1 - w.u0;
@@ -161,7 +488,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
     auto barrier = [&]() -> bool {
         return grid_barrier(a.bar, nbar++, GV_CONSUMERS, a.err, DERR_GRID_BARRIER_WAIT);
     };
-    auto token_rows = [&](const __nv_bfloat16* x, int K) -> GvX {
+    // Projection prologue: token rows into shared memory when they fit, RMSNorm scales.
+    auto token_rows = [&](const __nv_bfloat16* x, int K, const NormIn& nrm) -> GvX {
         GvX X;
         X.x = x;
         X.ldx = K;
@@ -169,7 +497,7 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
         X.K = K;
         X.Kp = cdiv(K, GV_BK) * GV_BK;
         X.xs = (long long)B * X.Kp * 2 <= a.xs_bytes ? reinterpret_cast<const __nv_bfloat16*>(xs_raw) : nullptr;
-        if (X.xs) gv_stage_x(reinterpret_cast<__nv_bfloat16*>(xs_raw), x, K, B, K, X.Kp);
+        gv_prologue(const_cast<__nv_bfloat16*>(X.xs), x, K, B, K, X.Kp, nrm, 0, rinv_s, rred_s);
         return X;
     };
     Epi base;
@@ -189,7 +517,7 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
         {
             Epi e = base;
             e.kind = EPI_QKV_ROPE;
-            e.pos0 = a.seq_len;
+            e.pos0 = s_len;  // this step's positions, already in shared memory
             e.rope_cos = a.rope_cos;
             e.rope_sin = a.rope_sin;
             e.H = a.H;
@@ -199,42 +527,14 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
             e.q_out = a.q;
             e.k_cache = kc;
             e.v_cache = vc;
-            const GvX X = token_rows(a.hw, D);
-            gv_rinv(ds_norm(a, nparts), B, 0, rinv_s, rred_s);
-            gv_consume<NB, EPI_QKV_ROPE>(ring, gv_work(nt_qkv, nku_D), X, Hd + 2 * Hkd, 0, rinv_s, e, a.ws,
+            const GvX X = token_rows(a.hw, D, ds_norm(a, nparts));
+            gv_consume<NB, EPI_QKV_ROPE, true>(ring, gv_work(nt_qkv, nku_D), X, Hd + 2 * Hkd, 0, rinv_s, e, a.ws,
                                          a.max_pieces[0], &last_s, a.err, DERR_MK_CONSUMER_WAIT);
             if (!barrier()) return;
         }
         // attention over the cache (the new token's K and V included)
-        {
-            AttnDecodeArgs aa;
-            aa.q = a.q;
-            aa.kc = kc;
-            aa.vc = vc;
-            aa.out = a.o;
-            aa.pos0 = a.seq_len;
-            aa.B = B;
-            aa.T = 1;
-            aa.H = a.H;
-            aa.Hk = a.Hk;
-            aa.d = a.d;
-            aa.S_max = a.S_max;
-            aa.n_splits = a.n_splits;
-            aa.tq = 1;
-            aa.n_qchunks = 1;
-            aa.ws_part = a.attn_part;
-            aa.ws_count = a.attn_cnt;
-            aa.scale_log2 = a.scale_log2;
-            aa.err = a.err;
-            const int items = B * a.Hk * a.n_splits;
-            for (int it = blockIdx.x; it < items; it += gridDim.x) {
-                const int grp = it / a.n_splits, split = it - grp * a.n_splits;
-                attn_split_item<__nv_bfloat16, RMAX, DS_NW, 16, 8>(aa, split, grp / a.Hk, grp % a.Hk, 0,
-                                                               reinterpret_cast<float*>(xs_raw), &last_s);
-                named_bar_sync(1, GV_CONSUMERS);  // the scratch is reused by the next item
-            }
-            if (!barrier()) return;
-        }
+        attn_consume(ring, a, l, asp, s_len, xs_raw);
+        if (!barrier()) return;
         // wo + residual; writes the ffn_norm input
         {
             Epi e = base;
@@ -245,9 +545,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
             e.wnext = a.norms[2 * l + 1];
             e.ss_out = a.ss;
             e.ss_out_ld = a.ss_ld;
-            const GvX X = token_rows(a.o, Hd);
-            gv_rinv(NormIn(), B, 0, rinv_s, rred_s);
-            gv_consume<NB, EPI_RESID>(ring, gv_work(nt_D, nku_Hd), X, D, 0, rinv_s, e, a.ws, a.max_pieces[1],
+            const GvX X = token_rows(a.o, Hd, NormIn());
+            gv_consume<NB, EPI_RESID, true>(ring, gv_work(nt_D, nku_Hd), X, D, 0, rinv_s, e, a.ws, a.max_pieces[1],
                                       &last_s, a.err, DERR_MK_CONSUMER_WAIT);
             nparts = resid_parts;
             if (!barrier()) return;
@@ -258,9 +557,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
             e.kind = EPI_SWIGLU;
             e.g_out = a.g;
             e.F = F;
-            const GvX X = token_rows(a.hw, D);
-            gv_rinv(ds_norm(a, nparts), B, 0, rinv_s, rred_s);
-            gv_consume<NB, EPI_SWIGLU>(ring, gv_work(nt_F, nku_D), X, F, 0, rinv_s, e, a.ws, a.max_pieces[2],
+            const GvX X = token_rows(a.hw, D, ds_norm(a, nparts));
+            gv_consume<NB, EPI_SWIGLU, true>(ring, gv_work(nt_F, nku_D), X, F, 0, rinv_s, e, a.ws, a.max_pieces[2],
                                        &last_s, a.err, DERR_MK_CONSUMER_WAIT);
             if (!barrier()) return;
         }
@@ -274,9 +572,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
             e.wnext = l + 1 < a.n_layers ? a.norms[2 * (l + 1)] : a.norms[2 * a.n_layers];
             e.ss_out = a.ss;
             e.ss_out_ld = a.ss_ld;
-            const GvX X = token_rows(a.g, F);
-            gv_rinv(NormIn(), B, 0, rinv_s, rred_s);
-            gv_consume<NB, EPI_RESID>(ring, gv_work(nt_D, nku_F), X, D, 0, rinv_s, e, a.ws, a.max_pieces[3],
+            const GvX X = token_rows(a.g, F, NormIn());
+            gv_consume<NB, EPI_RESID, true>(ring, gv_work(nt_D, nku_F), X, D, 0, rinv_s, e, a.ws, a.max_pieces[3],
                                       &last_s, a.err, DERR_MK_CONSUMER_WAIT);
             if (!barrier()) return;
         }
@@ -292,9 +589,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
         e.next_tok = a.next;
         e.seq_len = a.seq_len;
         e.advance = 1;
-        const GvX X = token_rows(a.hw, D);
-        gv_rinv(ds_norm(a, nparts), B, 0, rinv_s, rred_s);
-        gv_consume<NB, EPI_LOGITS>(ring, gv_work(nt_V, nku_D), X, a.vocab, 0, rinv_s, e, a.ws, a.max_pieces[4],
+        const GvX X = token_rows(a.hw, D, ds_norm(a, nparts));
+        gv_consume<NB, EPI_LOGITS, true>(ring, gv_work(nt_V, nku_D), X, a.vocab, 0, rinv_s, e, a.ws, a.max_pieces[4],
                                    &last_s, a.err, DERR_MK_CONSUMER_WAIT);
     } else {
         // layer stack only: hand out the hidden states and advance the cache lengths
@@ -322,41 +618,24 @@ static int pieces_for(int ntiles, int nku, int grid) {
 }
 
 static int hcdiv(int a, int b) { return (a + b - 1) / b; }
-static int rmax_of(int G) { return G <= 4 ? 4 : (G <= 8 ? 8 : 16); }
 
 DecodeStepPlan decode_step_plan(int B, int D, int H, int Hk, int d, int F, int vocab, int has_head, int max_keys,
                                 int num_sms, int smem_optin) {
+    (void)max_keys;
     DecodeStepPlan p = {};
     p.grid = num_sms;
     const int Hd = H * d, Hkd = Hk * d;
-    const int G = H / Hk;
     p.supported = B >= 1 && B <= 16 && D % 256 == 0 && Hd % GV_ROWS == 0 && Hkd % GV_ROWS == 0 && F % 8 == 0 &&
-                  d % 8 == 0 && d <= AD_DMAX && H % Hk == 0 && G <= 16;
+                  d == 128 && H % Hk == 0 && H / Hk <= 16;
     if (!p.supported) return p;
-    p.rmax = rmax_of(G);
-    // attention splits: minimise rounds x (per-round overhead + keys per split)
-    {
-        const int groups = B * Hk;
-        long long best = -1;
-        int best_ns = 1;
-        const int cap = hcdiv(max_keys, AD_GK) < AD_MAX_SPLITS ? hcdiv(max_keys, AD_GK) : AD_MAX_SPLITS;
-        for (int ns = 1; ns <= (cap > 1 ? cap : 1); ++ns) {
-            const long long rounds = ((long long)groups * ns + num_sms - 1) / num_sms;
-            const long long cost = rounds * (64 + hcdiv(max_keys, ns));
-            if (best < 0 || cost < best) {
-                best = cost;
-                best_ns = ns;
-            }
-        }
-        p.n_splits = best_ns;
-        p.attn_part_floats = (size_t)groups * G * best_ns * (d + 4);
-        p.attn_counters = (size_t)groups;
-    }
-    // shared memory: token-row copies that fit next to at least DS_MIN_STAGES ring
-    // stages, the attention scratch, and as many more stages as fit
+    const int R = H / Hk;
+    // attention: per (group, piece) records of 8 warps x 18 R floats; counters per (group, warp)
+    p.attn_part_floats = (size_t)B * Hk * num_sms * 8 * 18 * R;
+    p.attn_counters = (size_t)B * Hk * 8;
+    // shared memory: the query tile (4 KB), token-row copies that fit next to at
+    // least DS_MIN_STAGES ring stages, and as many more stages as fit
     const int avail = smem_optin - DS_SMEM_SLACK - 1024;  // 1 KB for the static shared variables
-    const int attn_bytes = attn_scratch_floats(p.rmax, DS_NW) * 4;
-    int xs = attn_bytes;
+    int xs = 4096;
     const int ks[3] = {D, Hd, F};
     for (int K : ks) {
         const int need = B * hcdiv(K, GV_BK) * GV_BK * 2;
@@ -390,12 +669,12 @@ DecodeStepPlan decode_step_plan(int B, int D, int H, int Hk, int d, int F, int v
     return p;
 }
 
-template <int NB, int RMAX>
+template <int NB>
 static cudaError_t launch_ds(const DecodeStepArgs& a, int smem, int grid, cudaStream_t s) {
     static int attr_smem = 0;
     if (attr_smem < smem) {
         const cudaError_t e =
-            cudaFuncSetAttribute(decode_step_kernel<NB, RMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            cudaFuncSetAttribute(decode_step_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         attr_smem = smem;
     }
@@ -405,25 +684,18 @@ static cudaError_t launch_ds(const DecodeStepArgs& a, int smem, int grid, cudaSt
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     // Cooperative: the launch fails rather than run if the CTAs cannot all be
-    // resident at once, which the grid barriers need.
+    // resident at once, which the grid barriers and the merges need.
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_step_kernel<NB, RMAX>, a);
+    return cudaLaunchKernelEx(&cfg, decode_step_kernel<NB>, a);
 }
 
 cudaError_t launch_decode_step(const DecodeStepArgs& a, const DecodeStepPlan& p, cudaStream_t s) {
     if (!p.supported || a.B < 1 || a.B > 16) return cudaErrorInvalidValue;
-    if (a.B <= 8) {
-        if (p.rmax == 4) return launch_ds<8, 4>(a, p.smem, p.grid, s);
-        if (p.rmax == 8) return launch_ds<8, 8>(a, p.smem, p.grid, s);
-        return launch_ds<8, 16>(a, p.smem, p.grid, s);
-    }
-    if (p.rmax == 4) return launch_ds<16, 4>(a, p.smem, p.grid, s);
-    if (p.rmax == 8) return launch_ds<16, 8>(a, p.smem, p.grid, s);
-    return launch_ds<16, 16>(a, p.smem, p.grid, s);
+    return a.B <= 8 ? launch_ds<8>(a, p.smem, p.grid, s) : launch_ds<16>(a, p.smem, p.grid, s);
 }
 
 }  // namespace lfw

@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(GV_THREADS, 2)
     __shared__ float rinv_s[16];
     __shared__ float rred_s[8][16];
     __shared__ int last_s;
-    GvRing ring{smem, full, full + GV_STAGES, GV_STAGES, 0, 0u};
+    GvRing ring{smem, full, full + GV_STAGES, GV_STAGES, 0, 0u, 0, 0};
     const int warp = threadIdx.x >> 5;
     const GvWork w = gv_work(ntiles, nku);
 
@@ -111,8 +111,7 @@ __global__ void __launch_bounds__(GV_THREADS, 2)
     X.K = a.K;
     X.Kp = nku * GV_BK;
     X.xs = (long long)a.M * X.Kp * 2 <= GV_XS_BYTES ? xs : nullptr;
-    if (X.xs) gv_stage_x(xs, a.x, a.ldx, a.M, a.K, X.Kp);
-    gv_rinv(a.epi.norm, a.M, a.m0, rinv_s, rred_s);
+    gv_prologue(const_cast<__nv_bfloat16*>(X.xs), a.x, a.ldx, a.M, a.K, X.Kp, a.epi.norm, a.m0, rinv_s, rred_s);
     gv_consume<NB, EPI>(ring, w, X, a.N, a.m0, rinv_s, a.epi, a.ws, max_pieces, &last_s, a.epi.err,
                         DERR_GEMV_CONSUMER_WAIT);
 }

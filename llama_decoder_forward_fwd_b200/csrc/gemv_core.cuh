@@ -14,9 +14,12 @@
 // empty mbarriers); eight consumer warps each own 16 of a tile's 128 rows and
 // consume every unit with mma.sync m16n8k16 (weights as the A operand, token
 // rows as B), so no reduction between warps is needed. A row tile whose k range
-// is split over several CTAs leaves one partial per CTA; the CTA that completes
-// the tile (atomic counter, no waiting) adds the partials in CTA order, which
-// keeps results deterministic, and its warps run the fused epilogue.
+// is split over several CTAs leaves one partial per CTA, added in CTA order (so
+// results are deterministic) by one CTA whose warps then run the fused epilogue:
+// in a launch that may not have all CTAs resident, the CTA that completes the
+// tile (atomic counter, no waiting); in the cooperative fused decode step, the
+// tile's first CTA (which reaches the tile last, at the end of its range), each
+// of its warps waiting for the other CTAs' pieces of its own 16 rows.
 //
 // Fragment layout: lane (g = lane/4, t = lane%4) reads 16 contiguous bf16 of its
 // rows g and g+8 at k0 + 16t. Because a dot product does not depend on the order
@@ -67,7 +70,23 @@ struct GvRing {
     int n;
     int st;
     uint32_t ph;
+    int inflight;     // producer: most copies in flight (issued, not landed); 0 = up to n
+    long long issued; // producer: copies issued so far
 };
+// Producer, before issuing a copy: with a limit on copies in flight, wait until
+// the copy issued `inflight` units ago has landed. Copies beyond the few that
+// keep HBM busy only lengthen the memory system's queues, and with them the
+// latency of every dependent load, atomic and fence of the consumers.
+DEVI bool ring_throttle(GvRing& r, uint32_t* err, uint32_t code) {
+    if (r.inflight <= 0 || r.inflight >= r.n || r.issued < r.inflight) return true;
+    int s = r.st - r.inflight;
+    uint32_t p = r.ph;
+    if (s < 0) {
+        s += r.n;
+        p ^= 1u;
+    }
+    return mbar_wait(&r.full[s], p, err, code);
+}
 DEVI void ring_next(GvRing& r) {
     if (++r.st == r.n) {
         r.st = 0;
@@ -111,6 +130,7 @@ DEVI bool gv_produce(GvRing& r, const GvWork& w, bool swiglu, const CUtensorMap*
     int tile = (int)(w.u0 / w.nku), kb = (int)(w.u0 % w.nku);  // tracked incrementally: no division in the loop
     for (long long u = w.u0; u < w.u1; ++u) {
         if (!mbar_wait(&r.empty[r.st], r.ph ^ 1u, err, code)) return false;
+        if (!ring_throttle(r, err, code)) return false;
         uint8_t* dst = r.stages + r.st * GV_UNIT_BYTES;
         const int kx = kb * GV_BK;
         mbar_arrive_expect_tx(&r.full[r.st], GV_UNIT_BYTES);
@@ -134,6 +154,7 @@ DEVI bool gv_produce(GvRing& r, const GvWork& w, bool swiglu, const CUtensorMap*
             kb = 0;
             ++tile;
         }
+        ++r.issued;
         ring_next(r);
     }
     return true;
@@ -157,27 +178,47 @@ DEVI void gv_drain(const GvRing& r, long long issued, uint32_t* err, uint32_t co
     }
 }
 
-// Consumers (256 threads): copy the M token rows of x (row stride ldx, K % 8 == 0)
-// into shared memory as [M][Kp], zero past K.
-DEVI void gv_stage_x(__nv_bfloat16* xs, const __nv_bfloat16* x, int ldx, int M, int K, int Kp) {
-    for (int i = threadIdx.x * 8; i < M * Kp; i += GV_CONSUMERS * 8) {
-        const int m = i / Kp, k = i - m * Kp;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (k < K) v = __ldcg(reinterpret_cast<const uint4*>(x + (size_t)m * ldx + k));
-        *reinterpret_cast<uint4*>(xs + i) = v;
-    }
-}
-
-// Consumers (256 threads): RMSNorm scale of each token row from the partial sums
-// of h^2 left by the producer of the input; 1 where the input is not normed.
-// Ends with a barrier of the consumers (which also publishes gv_stage_x).
-DEVI void gv_rinv(const NormIn& n, int M, int m0, float* rinv_s, float (*rred_s)[16]) {
+// Consumers (256 threads), at the start of a projection: copy the M token rows
+// of x (row stride ldx, K % 8 == 0) into shared memory as [M][Kp], zero past K
+// (when xs is not null), and compute each row's RMSNorm scale from the partial
+// sums of h^2 left by the producer of the input (1 where the input is not
+// normed). Every load of the first batch is issued before any is used, so the
+// prologue costs about one memory round trip. Ends with a barrier of the consumers.
+DEVI void gv_prologue(__nv_bfloat16* xs, const __nv_bfloat16* x, int ldx, int M, int K, int Kp, const NormIn& n,
+                      int m0, float* rinv_s, float (*rred_s)[16]) {
+    constexpr int XB = 8;  // 16-byte loads per thread per batch
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // partial sums: the first part of each row, loads only
     float part[16];
+    const bool has0 = n.ss != nullptr && (int)threadIdx.x < n.nparts;
 #pragma unroll
-    for (int m = 0; m < 16; ++m) part[m] = 0.f;
+    for (int m = 0; m < 16; ++m)
+        part[m] = (has0 && m < M) ? __ldcg(n.ss + (long long)threadIdx.x * n.ld + n.row0 + (long long)(m0 + m) * n.row_step)
+                                  : 0.f;
+    // token rows, XB loads in flight per thread
+    if (xs != nullptr) {
+        const int total = M * Kp;
+        for (int i0 = threadIdx.x * 8; i0 < total; i0 += GV_CONSUMERS * 8 * XB) {
+            uint4 v[XB];
+#pragma unroll
+            for (int j = 0; j < XB; ++j) {
+                const int i = i0 + j * GV_CONSUMERS * 8;
+                v[j] = make_uint4(0, 0, 0, 0);
+                if (i < total) {
+                    const int m = i / Kp, k = i - m * Kp;
+                    if (k < K) v[j] = __ldcg(reinterpret_cast<const uint4*>(x + (size_t)m * ldx + k));
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < XB; ++j) {
+                const int i = i0 + j * GV_CONSUMERS * 8;
+                if (i < total) *reinterpret_cast<uint4*>(xs + i) = v[j];
+            }
+        }
+    }
+    // remaining parts
     if (n.ss != nullptr)
-        for (int p = threadIdx.x; p < n.nparts; p += GV_CONSUMERS)
+        for (int p = threadIdx.x + GV_CONSUMERS; p < n.nparts; p += GV_CONSUMERS)
 #pragma unroll
             for (int m = 0; m < 16; ++m)
                 if (m < M) part[m] += __ldcg(n.ss + (long long)p * n.ld + n.row0 + (long long)(m0 + m) * n.row_step);
@@ -322,7 +363,7 @@ DEVI void gv_epilogue(int tile, const float (&c)[NB / 8][4], int N, int M, int m
 // tile reduction and the epilogues. A failed (timed-out) wait is recorded in
 // *err; the warp then stops waiting and runs the rest of its control flow on
 // whatever the stage holds, so every consumer warp still reaches every barrier.
-template <int NB, int EPI>
+template <int NB, int EPI, bool OWNER = false>
 DEVI bool gv_consume(GvRing& r, const GvWork& w, const GvX& X, int N, int m0, const float* rinv_s, const Epi& e,
                      const GemvScratch& ws, int max_pieces, int* last_s, uint32_t* err, uint32_t code) {
     constexpr int NM = NB / 8;
@@ -396,6 +437,54 @@ DEVI bool gv_consume(GvRing& r, const GvWork& w, const GvX& X, int N, int m0, co
         const long long cf = cta_of_unit(tu0, G, w.TU), cl = cta_of_unit(tu0 + w.nku - 1, G, w.TU);
         if (cf == cl) {
             gv_epilogue<NB, EPI>(tile, c, N, M, m0, rinv_s, e, ws, w.ntiles);
+        } else if (OWNER) {
+            // Every CTA of the tile but the first publishes its piece, one warp's rows
+            // at a time; the first CTA's warps wait for their rows' pieces.
+            float* base = ws.part + (size_t)tile * max_pieces * GV_PIECE_FLOATS + (warp * 32 + lane) * 8;
+            unsigned* cnt = ws.warp_cnt + tile * 8 + warp;
+            const long long pc = blockIdx.x - cf;
+            if (pc != 0) {
+                float* mine = base + (size_t)pc * GV_PIECE_FLOATS;
+#pragma unroll
+                for (int n = 0; n < NM; ++n)
+                    *reinterpret_cast<float4*>(mine + 4 * n) = make_float4(c[n][0], c[n][1], c[n][2], c[n][3]);
+                __syncwarp();
+                if (lane == 0) {
+                    __threadfence();
+                    atomicAdd(cnt, 1u);
+                }
+                __syncwarp();
+            } else {
+                if (lane == 0) {
+                    const unsigned want = (unsigned)(cl - cf);
+                    if (ok && ld_acquire_gpu(cnt) < want) {
+                        const uint64_t t0 = globaltimer();
+                        while (ld_acquire_gpu(cnt) < want) {
+                            if (globaltimer() - t0 > kWaitLimitNs) {
+                                atomicCAS(err, 0u, code);
+                                break;
+                            }
+                        }
+                    }
+                    *cnt = 0u;
+                }
+                __syncwarp();
+                float t[NM][4];
+#pragma unroll
+                for (int n = 0; n < NM; ++n) t[n][0] = c[n][0], t[n][1] = c[n][1], t[n][2] = c[n][2], t[n][3] = c[n][3];
+                for (long long p = 1; p <= cl - cf; ++p) {
+                    const float* src = base + (size_t)p * GV_PIECE_FLOATS;
+#pragma unroll
+                    for (int n = 0; n < NM; ++n) {
+                        const float4 v = __ldcg(reinterpret_cast<const float4*>(src + 4 * n));
+                        t[n][0] += v.x;
+                        t[n][1] += v.y;
+                        t[n][2] += v.z;
+                        t[n][3] += v.w;
+                    }
+                }
+                gv_epilogue<NB, EPI>(tile, t, N, M, m0, rinv_s, e, ws, w.ntiles);
+            }
         } else {
             float* base = ws.part + (size_t)tile * max_pieces * GV_PIECE_FLOATS;
             float* mine = base + (size_t)(blockIdx.x - cf) * GV_PIECE_FLOATS + (warp * 32 + lane) * 8;

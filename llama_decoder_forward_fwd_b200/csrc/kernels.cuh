@@ -90,6 +90,8 @@ struct GemvScratch {
     int tiles_cap = 0;
     unsigned long long* am_best = nullptr;  // [16] packed (logit, id) maxima
     unsigned* done_cnt = nullptr;           // [1] tiles finished (argmax)
+    unsigned* warp_cnt = nullptr;           // [tiles_cap * 8] pieces published per (tile, warp)
+                                            // (fused decode step: the tile's owner waits for them)
 };
 struct GemvPlan {
     int ntiles, nkb, grid, max_pieces;
@@ -175,8 +177,9 @@ struct DecodeStepArgs {
     int B = 0, D = 0, H = 0, Hk = 0, d = 0, F = 0, vocab = 0, S_max = 0, n_layers = 0;
     float eps = 0.f, scale_log2 = 0.f;
     int has_head = 0;
-    int n_splits = 1;                // attention key splits
-    int n_stages = 0, xs_bytes = 0;  // shared memory: ring stages; token rows / attention scratch
+    int n_stages = 0, xs_bytes = 0;  // shared memory: ring stages; token rows / query tile
+    int prefetch_units = 0;          // units the producer prefetches into L2 ahead of its loads
+    int inflight_units = 0;          // most units in flight per CTA (0: the whole ring)
     int max_pieces[5] = {1, 1, 1, 1, 1};  // split-tile slots of QKV, wo, w1/w3, w2, lm_head
     // inputs and outputs of the step
     const int32_t* tok = nullptr;  // [B] token ids (models with embedding and head)
@@ -185,13 +188,15 @@ struct DecodeStepArgs {
     int32_t* next = nullptr;       // [B] greedy next tokens
     float* logits = nullptr;       // [B][vocab] or nullptr
     // weights
-    const CUtensorMap* tmaps = nullptr;  // device: TM_PER_LAYER maps per layer, then the lm_head map
+    const CUtensorMap* tmaps = nullptr;  // device: TM_PER_LAYER maps per layer, then the lm_head map,
+                                         // then the K and V cache maps (box 64 dims x 32 rows)
     const void* const* norms = nullptr;  // device: attention_norm[l], ffn_norm[l] per layer, then the final norm
     const void* tok_emb = nullptr;
     // state and activations (layouts as above)
     void* kc = nullptr;
     void* vc = nullptr;
-    long long layer_elems = 0;
+    long long layer_elems = 0;        // elements of one layer's K (or V) cache
+    long long kv_rows_per_layer = 0;  // its rows of head_dim elements
     int32_t* seq_len = nullptr;
     float* h = nullptr;
     __nv_bfloat16* hw = nullptr;
@@ -204,14 +209,14 @@ struct DecodeStepArgs {
     const float* rope_sin = nullptr;
     // scratch (counters zero between launches; *bar zeroed before each launch)
     GemvScratch ws;
-    float* attn_part = nullptr;
-    unsigned* attn_cnt = nullptr;
+    float* attn_part = nullptr;  // per (group, piece, warp): O[R][16], m[R], l[R]
+    unsigned* attn_cnt = nullptr;  // per (group, warp), zero between launches
     unsigned* bar = nullptr;
     uint32_t* err = nullptr;
 };
 struct DecodeStepPlan {
     bool supported;
-    int grid, rmax, n_splits, n_stages, xs_bytes, smem;
+    int grid, n_stages, xs_bytes, smem;
     int max_pieces[5];
     size_t part_floats;  // split-tile partial floats needed
     int tiles;           // tile counters needed

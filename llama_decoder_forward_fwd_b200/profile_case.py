@@ -11,6 +11,8 @@
     python -m llama_decoder_forward_fwd_b200.profile_case decode-head
         the lm_head + argmax of the Llama-3-8B shape on one token (1.05 GB)
 
+A trailing --fused runs the decode steps as the fused single-launch kernel.
+
 Weights are seeded random (the bench's distributions); nothing is checked here.
 """
 import sys
@@ -20,12 +22,15 @@ import torch
 import llama_decoder_forward_fwd_b200 as L
 
 
+FLAGS = L.LLM_FLAG_FUSED_DECODE if "--fused" in sys.argv[2:] else 0
+
+
 def _layer_model(prefill_tokens, S_max=4096, has_head=False, vocab=128256):
     import seeded_inputs as S
     shape = S.WORKLOADS["llama3-8b-bf16-b1-p2048-g256"].shape.replace(
         n_layers=1, has_embed_and_head=has_head, max_seq_len=S_max, vocab=vocab)
     glob, layers = S.make_weights(shape, 1234, device="cuda")
-    return shape, L.Model(shape, glob, layers, max_batch=1, max_tokens=max(prefill_tokens, 1))
+    return shape, L.Model(shape, glob, layers, max_batch=1, max_tokens=max(prefill_tokens, 1), flags=FLAGS)
 
 
 def decode_layer():

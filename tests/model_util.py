@@ -20,9 +20,8 @@ def rel_l2(a, b) -> float:
 
 
 def build_pair(shape, seed, batch, max_tokens=0, flags=0, taps=True):
-    """GPU model and oracle on the same weights. With taps the GPU model keeps every
-    layer's output (which runs decode steps layer by layer); without, bf16 decode
-    steps run as the fused single-launch kernel."""
+    """GPU model and oracle on the same weights; with taps the GPU model keeps every
+    layer's output (llm_debug_tap)."""
     glob, layers = S.make_weights(shape, seed)
     model = L.Model(shape, glob, layers, max_batch=batch, max_tokens=max_tokens,
                     flags=flags | (L.LLM_FLAG_DEBUG_TAPS if taps else 0))
