@@ -235,7 +235,7 @@ def run_ours(args, rank, world, local_rank):
 
     glob, layers = S.make_weights(shape, w.seed, device=dev)
     stream = torch.cuda.Stream(device=dev)
-    extra = L.LLM_FLAG_FUSED_DECODE if args.fused else 0
+    extra = (L.LLM_FLAG_FUSED_DECODE if args.fused else 0) | (L.LLM_FLAG_PDL if args.pdl else 0)
     model = L.Model(shape, glob, layers, max_batch=B, max_tokens=B * T,
                     flags=extra | (0 if args.no_graph else L.LLM_FLAG_CUDA_GRAPH), stream=stream, device=dev)
     prompt = S.make_tokens(w.seed, B, T, shape.vocab).to(dev)
@@ -372,7 +372,7 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": WORKLOAD, "batch": B, "prompt_len": T, "decode_steps": G,
                    "layers": shape.n_layers, "dim": shape.dim, "vocab": shape.vocab,
                    "l2": "inputs larger than L2: every step streams 16 GB of weights",
-                   "cuda_graph_decode": not args.no_graph, "decode_kernel": "fused step" if fused else "layerwise",
+                   "cuda_graph_decode": not args.no_graph, "decode_kernel": "fused step" if fused else "layerwise", "pdl": bool(args.pdl),
                    "parallelism": f"replicas x{world}"},
         "prefill": prefill, "decode": decode, "roofline": roof, "kernels": kernel_table,
         "cpu_baseline": ({k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")} if cpu else None),
@@ -392,6 +392,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--pdl", action="store_true",
+                    help="programmatic dependent launch between consecutive kernels")
     ap.add_argument("--fused", action="store_true",
                     help="decode each step as the fused single-launch kernel instead of one launch per "
                          "projection and attention")

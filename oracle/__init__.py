@@ -36,6 +36,13 @@ Sources (page title, then section), all restated in this module's own words:
 * "LLaMA2" (downcodes): RoPE as a rotation whose q.k product depends only on the
   position offset; GQA/MQA share K/V heads among query heads; the KV cache.
 
+``OracleModel(..., bf16_activations=True)`` is the same computation with the
+activations rounded to bf16 (nearest, ties to even) at the points where a bf16
+implementation stores them: each projection input h * norm weight (the norm's
+1/rms scale applied after the product), q, k and v after RoPE, the attention
+output and the SwiGLU output. It exists to state what that storage policy alone
+does to the result at depth; every other value stays exact.
+
 Readings where the pages are silent or garbled (each is also listed in the
 design notes): RoPE rotates interleaved adjacent pairs (2i, 2i+1) with angle
 p * theta^(-2i/d); the score scale is 1/sqrt(head_dim); masked scores are -inf
@@ -52,7 +59,7 @@ import numpy as np
 import torch
 
 __all__ = [
-    "f64", "rmsnorm", "rope_tables", "rope", "softmax", "silu", "attention",
+    "f64", "round_bf16", "rmsnorm", "rope_tables", "rope", "softmax", "silu", "attention",
     "swiglu_ffn", "argmax_first", "OracleModel",
 ]
 
@@ -62,6 +69,19 @@ def f64(t) -> np.ndarray:
     if isinstance(t, torch.Tensor):
         return t.detach().to("cpu").to(torch.float64).numpy()
     return np.asarray(t, dtype=np.float64)
+
+
+def round_bf16(x) -> np.ndarray:
+    """Round to the nearest value with an 8-bit significand (bf16), ties to even.
+
+    With x = m * 2^e and 0.5 <= |m| < 1, the nearest such value is
+    rint(m * 2^8) * 2^(e - 8), where rint rounds halves to even. (bf16 keeps 8
+    significant bits, 7 of them stored; subnormals and overflow do not arise for
+    the activations this is used on.)
+    """
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)
+    return np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)
 
 
 def rmsnorm(x: np.ndarray, w: np.ndarray, eps: float) -> np.ndarray:
@@ -173,8 +193,10 @@ class OracleModel:
     K[l][b] has shape [n_pos, Hk, d].
     """
 
-    def __init__(self, shape, glob: Dict, layers, batch: int, keep_f64_layers: bool = True):
+    def __init__(self, shape, glob: Dict, layers, batch: int, keep_f64_layers: bool = True,
+                 bf16_activations: bool = False):
         self.s = shape
+        self.bf16 = bf16_activations
         self.glob = glob
         self._layers = layers
         self._cache64: Dict[int, Dict[str, np.ndarray]] = {}
@@ -226,23 +248,35 @@ class OracleModel:
         w = self.layer(l)
         B, T, D = h.shape
         H, Hk, d = s.n_heads, s.n_kv_heads, s.head_dim
-        x = rmsnorm(h, w["attention_norm"], s.norm_eps)
+        r = self._round
+        x = self._norm_in(h, w["attention_norm"])
         out = np.empty((B, T, H * d))
         for b in range(B):
             pos = pos0[b] + np.arange(T)
             q = (x[b] @ w["wq"].T).reshape(T, H, d)
             k = (x[b] @ w["wk"].T).reshape(T, Hk, d)
-            v = (x[b] @ w["wv"].T).reshape(T, Hk, d)
-            q = rope(q, pos, s.rope_theta)
-            k = rope(k, pos, s.rope_theta)
+            v = r((x[b] @ w["wv"].T).reshape(T, Hk, d))
+            q = r(rope(q, pos, s.rope_theta))
+            k = r(rope(k, pos, s.rope_theta))
             assert self.K[l][b].shape[0] == pos0[b], "cache length and position disagree"
             self.K[l][b] = np.concatenate([self.K[l][b], k], axis=0)
             self.V[l][b] = np.concatenate([self.V[l][b], v], axis=0)
             kpos = np.arange(self.K[l][b].shape[0])
-            out[b] = attention(q, self.K[l][b], self.V[l][b], pos, kpos)
+            out[b] = r(attention(q, self.K[l][b], self.V[l][b], pos, kpos))
         h = h + out @ w["wo"].T
-        x = rmsnorm(h, w["ffn_norm"], s.norm_eps)
-        return h + swiglu_ffn(x, w["w1"], w["w3"], w["w2"])
+        x = self._norm_in(h, w["ffn_norm"])
+        return h + r(silu(x @ w["w1"].T) * (x @ w["w3"].T)) @ w["w2"].T
+
+    def _round(self, a: np.ndarray) -> np.ndarray:
+        return round_bf16(a) if self.bf16 else a
+
+    def _norm_in(self, h: np.ndarray, wn: np.ndarray) -> np.ndarray:
+        """RMSNorm(h) * wn; with bf16 activations, h * wn is stored in bf16 and the
+        1/rms scale is applied to it afterwards (the same value in exact arithmetic)."""
+        if not self.bf16:
+            return rmsnorm(h, wn, self.s.norm_eps)
+        rinv = 1.0 / np.sqrt(np.mean(h * h, axis=-1, keepdims=True) + self.s.norm_eps)
+        return round_bf16(h * wn) * rinv
 
     # ---- whole passes --------------------------------------------------
     def _run_layers(self, h: np.ndarray, taps: Optional[List[np.ndarray]]):
@@ -258,7 +292,7 @@ class OracleModel:
 
     def logits_last(self, h: np.ndarray) -> np.ndarray:
         """Final RMSNorm of the last position, then logits = x @ output^T ("Linear")."""
-        x = rmsnorm(h[:, -1, :], f64(self.glob["norm"]), self.s.norm_eps)
+        x = self._norm_in(h[:, -1, :], f64(self.glob["norm"]))
         return x @ self.lm_head().T
 
     def prefill(self, tokens, taps: Optional[List[np.ndarray]] = None):

@@ -323,3 +323,52 @@ def test_page_printed_tiny_config():
     assert (w.shape.dim, w.shape.n_layers, w.shape.n_heads, w.shape.vocab, w.shape.max_seq_len,
             w.decode_steps) == (gold["dim"], gold["n_layers"], gold["n_heads"], gold["vocab_size"],
                                 gold["max_seq_len"], gold["max_new_tokens"])
+
+
+# ---- bf16 storage emulation ---------------------------------------------------
+def test_round_bf16_definition():
+    """Nearest value with an 8-bit significand, ties to even; against the definition,
+    hand-worked ties, the half-ulp bound, and torch's float32 -> bfloat16 cast."""
+    r = O.round_bf16
+    exact = np.array([0.0, 1.0, -1.5, 3.25, 2.0 ** -20, -(2.0 ** 30), 1 + 2.0 ** -7])
+    assert np.array_equal(r(exact), exact)
+    # ties: 1 + 2^-8 lies halfway between 1 and 1 + 2^-7 -> even significand (1.0);
+    # 1 + 3 * 2^-8 lies halfway between 1 + 2^-7 and 1 + 2^-6 -> 1 + 2^-6
+    assert r(1 + 2.0 ** -8) == 1.0
+    assert r(1 + 3 * 2.0 ** -8) == 1 + 2.0 ** -6
+    assert r(-(1 + 2.0 ** -8)) == -1.0
+    assert r(1 + 2.0 ** -8 + 2.0 ** -30) == 1 + 2.0 ** -7   # just above the tie
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal(100000) * np.exp(rng.uniform(-20, 20, 100000))
+    y = r(x)
+    assert np.all(np.abs(y - x) <= 2.0 ** -8 * np.abs(x))           # half an ulp
+    m, _ = np.frexp(y)
+    assert np.all(np.ldexp(m, 8) == np.rint(np.ldexp(m, 8)))         # 8 significant bits
+    x32 = x.astype(np.float32)
+    ref = torch.from_numpy(x32).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(r(x32.astype(np.float64)), ref)
+
+
+def test_bf16_emulation_rounds_where_stated_and_stays_close():
+    shape = S.ModelShape(dim=64, n_layers=2, n_heads=4, n_kv_heads=2, head_dim=16, ffn_hidden=96,
+                         vocab=50, max_seq_len=32, norm_eps=1e-5, rope_theta=10000.0, dtype="bf16",
+                         tie_embeddings=False)
+    glob, layers = S.make_weights(shape, 11)
+    tok = S.make_tokens(11, 2, 9, shape.vocab).numpy()
+    plain = O.OracleModel(shape, glob, layers, 2)
+    emu = O.OracleModel(shape, glob, layers, 2, bf16_activations=True)
+    same = O.OracleModel(shape, glob, layers, 2, bf16_activations=False)
+    tp, te, ts = [], [], []
+    _, lp = plain.prefill(tok, tp)
+    _, le = emu.prefill(tok, te)
+    _, ls = same.prefill(tok, ts)
+    assert np.array_equal(lp, ls) and all(np.array_equal(a, b) for a, b in zip(tp, ts))
+    for l in range(shape.n_layers):
+        for b in range(2):
+            assert np.array_equal(O.round_bf16(emu.K[l][b]), emu.K[l][b])
+            assert np.array_equal(O.round_bf16(emu.V[l][b]), emu.V[l][b])
+            assert not np.array_equal(O.round_bf16(plain.K[l][b]), plain.K[l][b])
+        d = np.linalg.norm(te[l] - tp[l]) / np.linalg.norm(tp[l])
+        assert 1e-5 < d < 1e-2, d
+    d = np.linalg.norm(le - lp) / np.linalg.norm(lp)
+    assert 1e-5 < d < 1e-2, d
