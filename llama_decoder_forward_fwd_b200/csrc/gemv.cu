@@ -89,16 +89,13 @@ __global__ void __launch_bounds__(GV_THREADS, 2)
         tma_prefetch_desc(&tm2);
     }
     __syncthreads();
+    pdl_trigger();
 
     if (warp == 8) {
-        // producer: weights do not depend on the previous kernel. With programmatic
-        // dependent launch, the next kernel may start once every CTA has issued its
-        // last copy, so its producer streams while this kernel drains (triggering at
-        // the start instead lets several kernels pile onto the SMs at once).
+        // producer: weights do not depend on the previous kernel
         if ((threadIdx.x & 31) == 0) {
             const bool ok = gv_produce(ring, w, EPI == EPI_SWIGLU, &tm0, &tm1, &tm2, a.seg_rows[0], a.seg_rows[1],
                                        a.epi.err, DERR_GEMV_PRODUCER_WAIT);
-            pdl_trigger();
             gv_drain(ring, ok ? w.u1 - w.u0 : GV_STAGES, a.epi.err, DERR_GEMV_PRODUCER_WAIT);
         }
         pdl_wait();
