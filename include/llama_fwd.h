@@ -235,7 +235,9 @@ int llm_op_gemm_bf16(const void* A, const void* B, float* C, int M, int N, int K
  * [M, N]. Needs K % 8 == 0. workspace: device scratch of at least
  * llm_op_gemv_workspace(N, K) bytes, 16-byte aligned, contents arbitrary (the
  * call clears the part it needs); calls sharing one workspace must not overlap
- * in time. Source: the per-token projection q_per_token = x @ wq_head^T of
+ * in time. The kernel is launched cooperatively (one CTA per SM, all resident
+ * at once); where the device cannot host that, the call returns LLM_ERR_CUDA.
+ * Source: the per-token projection q_per_token = x @ wq_head^T of
  * "Building llama3 from scratch", for the decode phase of llama3.np "Generasi".
  */
 size_t llm_op_gemv_workspace(int N, int K);

@@ -1107,13 +1107,15 @@ static size_t gemv_ws_layout(int N, int K, size_t* off_part, GemvScratch* ws, vo
     const int tiles = gemv_num_tiles(EPI_STORE_F32, N);
     const size_t pf = gemv_scratch_floats(EPI_STORE_F32, N, K, sms);
     const size_t o_cnt = 0;
-    const size_t o_best = (o_cnt + (size_t)tiles * 4 + 255) & ~size_t(255);
+    const size_t o_wcnt = (o_cnt + (size_t)tiles * 4 + 255) & ~size_t(255);
+    const size_t o_best = (o_wcnt + (size_t)tiles * 8 * 4 + 255) & ~size_t(255);
     const size_t o_done = o_best + 256;
     const size_t o_part = o_done + 256;
     if (off_part) *off_part = o_part;
     if (ws && base) {
         char* b = reinterpret_cast<char*>(base);
         ws->tile_cnt = reinterpret_cast<unsigned*>(b + o_cnt);
+        ws->warp_cnt = reinterpret_cast<unsigned*>(b + o_wcnt);
         ws->tiles_cap = tiles;
         ws->am_best = reinterpret_cast<unsigned long long*>(b + o_best);
         ws->done_cnt = reinterpret_cast<unsigned*>(b + o_done);

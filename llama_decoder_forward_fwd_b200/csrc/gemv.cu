@@ -55,7 +55,10 @@ DEVI void logits_finish(const Epi& e, int M, int ntiles, int* last_s) {
 }
 
 
-// bf16 projection: one CTA per SM, GV_STAGES units in flight per CTA.
+// bf16 projection: one CTA per SM, GV_STAGES units in flight per CTA. The launch is
+// cooperative (every CTA resident), so a row tile split over several CTAs is
+// finished by its first CTA, which waits for the other CTAs' pieces; they publish
+// them as soon as they reach the end of their part and move on.
 constexpr int GV_STAGES = 5;                    // ~110 KB per CTA: two CTAs (of consecutive
                                                 // launches) can share an SM
 constexpr int GV_THREADS = GV_CONSUMERS + 32;   // 8 consumer warps + 1 producer warp
@@ -112,8 +115,8 @@ __global__ void __launch_bounds__(GV_THREADS, 2)
     X.Kp = nku * GV_BK;
     X.xs = (long long)a.M * X.Kp * 2 <= GV_XS_BYTES ? xs : nullptr;
     gv_prologue(const_cast<__nv_bfloat16*>(X.xs), a.x, a.ldx, a.M, a.K, X.Kp, a.epi.norm, a.m0, rinv_s, rred_s);
-    gv_consume<NB, EPI>(ring, w, X, a.N, a.m0, rinv_s, a.epi, a.ws, max_pieces, &last_s, a.epi.err,
-                        DERR_GEMV_CONSUMER_WAIT);
+    gv_consume<NB, EPI, true>(ring, w, X, a.N, a.m0, rinv_s, a.epi, a.ws, max_pieces, &last_s, a.epi.err,
+                              DERR_GEMV_CONSUMER_WAIT);
 }
 
 // fp32 kernel (CUDA cores): a warp owns a pair of logical rows, a CTA 8 pairs.
@@ -245,21 +248,33 @@ __global__ void __launch_bounds__(GEMV_THREADS) gemv_f32_kernel(const GemvArgs<f
 // ---------------------------------------------------------------- launchers
 template <int NB, int EPI>
 static cudaError_t launch_bf16_e(const GemvArgs<__nv_bfloat16>& a, cudaStream_t s, bool pdl) {
-    static bool attr = false;
-    if (!attr) {
+    static bool smem_set = false;
+    if (!smem_set) {
         cudaError_t e = cudaFuncSetAttribute(gemv_bf16_kernel<NB, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM);
         if (e != cudaSuccess) return e;
-        attr = true;
+        smem_set = true;
     }
     if (!a.tmw[0]) return cudaErrorInvalidValue;
     const GemvPlan p = gemv_plan(EPI, a.N, a.K, a.num_sms, 1);
     if ((size_t)p.ntiles * p.max_pieces * GV_PIECE_FLOATS > a.ws.part_floats || p.ntiles > a.ws.tiles_cap)
         return cudaErrorInvalidValue;
+    if (!a.ws.warp_cnt) return cudaErrorInvalidValue;
     const CUtensorMap& m0 = *a.tmw[0];
     const CUtensorMap& m1 = a.tmw[1] ? *a.tmw[1] : m0;
     const CUtensorMap& m2 = a.tmw[2] ? *a.tmw[2] : m0;
-    return launch_k(gemv_bf16_kernel<NB, EPI>, dim3(p.grid), GV_THREADS, GV_SMEM, s, pdl, m0, m1, m2, a, p.ntiles,
-                    p.nkb, p.max_pieces);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.grid);
+    cfg.blockDim = dim3(GV_THREADS);
+    cfg.dynamicSmemBytes = GV_SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, gemv_bf16_kernel<NB, EPI>, m0, m1, m2, a, p.ntiles, p.nkb, p.max_pieces);
 }
 
 template <int NB>
