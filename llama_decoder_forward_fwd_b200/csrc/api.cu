@@ -143,8 +143,6 @@ struct llm_model {
     // pointers, and the grid-barrier counter
     bool fused = false;
     int smem_optin = 0;
-    int fused_prefetch = 0;  // L2 prefetch distance of the fused step (LLM_FUSED_PREFETCH_UNITS)
-    int fused_inflight = 0;  // weight copies in flight per SM (LLM_FUSED_INFLIGHT_UNITS)
     CUtensorMap* d_tmaps = nullptr;
     const void** d_norms = nullptr;
     unsigned* ds_bar = nullptr;
@@ -562,8 +560,6 @@ int run_fused_step(llm_model* m, int B, const int32_t* tok, const float* h_in, f
     a.has_head = c.has_embed_and_head;
     a.n_stages = p.n_stages;
     a.xs_bytes = p.xs_bytes;
-    a.prefetch_units = m->fused_prefetch;
-    a.inflight_units = m->fused_inflight;
     for (int i = 0; i < 5; ++i) a.max_pieces[i] = p.max_pieces[i];
     a.tok = tok;
     a.h_in = h_in;
@@ -747,7 +743,6 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
         m->gws.part_floats = pf;
         m->gws.tiles_cap = tiles;
         MALLOC_OR_BAIL(m->gws.part, pf * 4);
-        MALLOC_OR_BAIL(m->gws.tile_cnt, (size_t)tiles * 4);
         MALLOC_OR_BAIL(m->gws.am_best, 16 * 8);
         MALLOC_OR_BAIL(m->gws.done_cnt, 16);
         MALLOC_OR_BAIL(m->gws.warp_cnt, (size_t)tiles * 8 * 4);
@@ -764,8 +759,7 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
         cudaMemsetAsync(m->seq_len, 0, (size_t)c.max_batch * 4, m->stream) != cudaSuccess ||
         cudaMemsetAsync(m->d_err, 0, 64, m->stream) != cudaSuccess ||
         cudaMemsetAsync(m->ss, 0, (size_t)parts * Mx * 4, m->stream) != cudaSuccess ||
-        (m->bf16 && (cudaMemsetAsync(m->gws.tile_cnt, 0, (size_t)m->gws.tiles_cap * 4, m->stream) != cudaSuccess ||
-                     cudaMemsetAsync(m->gws.am_best, 0, 16 * 8, m->stream) != cudaSuccess ||
+        (m->bf16 && (cudaMemsetAsync(m->gws.am_best, 0, 16 * 8, m->stream) != cudaSuccess ||
                      cudaMemsetAsync(m->gws.done_cnt, 0, 16, m->stream) != cudaSuccess ||
                      cudaMemsetAsync(m->gws.warp_cnt, 0, (size_t)m->gws.tiles_cap * 8 * 4, m->stream) != cudaSuccess)))
         return bail(fail(LLM_ERR_CUDA, "cudaMemsetAsync failed"));
@@ -827,11 +821,9 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
                 m->gws.part_floats = pf;
             }
             if (tiles > m->gws.tiles_cap) {
-                MALLOC_OR_BAIL(m->gws.tile_cnt, (size_t)tiles * 4);
                 MALLOC_OR_BAIL(m->gws.warp_cnt, (size_t)tiles * 8 * 4);
                 m->gws.tiles_cap = tiles;
-                if (cudaMemsetAsync(m->gws.tile_cnt, 0, (size_t)tiles * 4, m->stream) != cudaSuccess ||
-                    cudaMemsetAsync(m->gws.warp_cnt, 0, (size_t)tiles * 8 * 4, m->stream) != cudaSuccess)
+                if (cudaMemsetAsync(m->gws.warp_cnt, 0, (size_t)tiles * 8 * 4, m->stream) != cudaSuccess)
                     return bail(fail(LLM_ERR_CUDA, "cudaMemsetAsync failed"));
             }
             if (af > m->attn_ws_floats) {
@@ -872,10 +864,6 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
                 cudaMemsetAsync(m->ds_bar, 0, 64, m->stream) != cudaSuccess)
                 return bail(fail(LLM_ERR_CUDA, "fused decode step setup copies failed"));
             m->fused = true;
-            if (const char* pe = getenv("LLM_FUSED_PREFETCH_UNITS")) m->fused_prefetch = atoi(pe);
-            if (m->fused_prefetch < 0) m->fused_prefetch = 0;
-            if (const char* ie = getenv("LLM_FUSED_INFLIGHT_UNITS")) m->fused_inflight = atoi(ie);
-            if (m->fused_inflight < 0) m->fused_inflight = 0;
         }
     }
     if (cudaStreamSynchronize(m->stream) != cudaSuccess) return bail(fail(LLM_ERR_CUDA, "init sync failed"));
@@ -1106,15 +1094,13 @@ static size_t gemv_ws_layout(int N, int K, size_t* off_part, GemvScratch* ws, vo
     const int sms = num_sms_current();
     const int tiles = gemv_num_tiles(EPI_STORE_F32, N);
     const size_t pf = gemv_scratch_floats(EPI_STORE_F32, N, K, sms);
-    const size_t o_cnt = 0;
-    const size_t o_wcnt = (o_cnt + (size_t)tiles * 4 + 255) & ~size_t(255);
+    const size_t o_wcnt = 0;
     const size_t o_best = (o_wcnt + (size_t)tiles * 8 * 4 + 255) & ~size_t(255);
     const size_t o_done = o_best + 256;
     const size_t o_part = o_done + 256;
     if (off_part) *off_part = o_part;
     if (ws && base) {
         char* b = reinterpret_cast<char*>(base);
-        ws->tile_cnt = reinterpret_cast<unsigned*>(b + o_cnt);
         ws->warp_cnt = reinterpret_cast<unsigned*>(b + o_wcnt);
         ws->tiles_cap = tiles;
         ws->am_best = reinterpret_cast<unsigned long long*>(b + o_best);

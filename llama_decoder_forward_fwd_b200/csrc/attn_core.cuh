@@ -252,13 +252,11 @@ DEVI void attn_split_item(const AttnDecodeArgs& a, int split, int b, int kvh, in
     // The last split of this group merges all splits.
     named_bar_sync(1, NT);
     if (threadIdx.x == 0) {
-        __threadfence();
-        const unsigned prev = atomicAdd(a.ws_count + grp, 1u);
+        const unsigned prev = atom_add_acq_rel(a.ws_count + grp, 1u);
         *last_s = (prev == (unsigned)(a.n_splits - 1));
     }
     named_bar_sync(1, NT);
     if (!*last_s) return;
-    __threadfence();
     const int ns = a.n_splits;
     for (int idx = threadIdx.x; idx < R * ns; idx += NT) {
         const int r = idx / ns, sp = idx % ns;

@@ -88,6 +88,24 @@ DEVI bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err, uint32_t code
     }
 }
 
+// Release increment: every write that happens before it (this thread's, and the
+// writes of other threads ordered before it by a CTA or warp barrier) is visible
+// to a thread that observes the new count with an acquire load. It orders only
+// what a publish needs, unlike a full fence followed by an atomic.
+DEVI void red_release_add(unsigned* p, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Acquire-release increment returning the previous count: publishes this
+// thread's earlier writes (and those ordered before it by a barrier) and, for the
+// thread that sees the final count, makes every earlier publisher's writes
+// visible to what follows it.
+DEVI unsigned atom_add_acq_rel(unsigned* p, unsigned v) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 DEVI unsigned ld_acquire_gpu(const unsigned* p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -98,16 +116,15 @@ DEVI unsigned ld_acquire_gpu(const unsigned* p) {
 // threads of every CTA (the CTA's other warps do not take part). Barrier number
 // `index` (0, 1, 2, ...) of the launch waits until every CTA has arrived
 // `index + 1` times (*count is zero at launch). Writes made before the barrier
-// by any CTA are visible to every thread after it (release fence + arrival,
-// acquire polling, CTA barrier). The wait is bounded: on timeout it records
+// by any CTA are visible to every thread after it (CTA barrier, release
+// arrival, acquire polling, CTA barrier). The wait is bounded: on timeout it records
 // `code` in *err and returns false; it also returns false as soon as *err
 // holds another CTA's error, so all CTAs leave promptly.
 DEVI bool grid_barrier(unsigned* count, unsigned index, int nthreads, uint32_t* err, uint32_t code) {
     __shared__ int gb_ok;
     named_bar_sync(1, nthreads);
     if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(count, 1u);
+        red_release_add(count, 1u);
         const unsigned target = (index + 1) * gridDim.x;
         int ok = 1;
         if (ld_acquire_gpu(count) < target) {

@@ -117,7 +117,6 @@ DEVI bool attn_produce(GvRing& r, const DecodeStepArgs& a, int l, const AttnSpli
     int n = sp.u0 < sp.u1 ? group_units(s_len, gr, a.Hk) : 0;
     for (long long u = sp.u0; u < sp.u1; ++u) {
         if (!mbar_wait(&r.empty[r.st], r.ph ^ 1u, a.err, DERR_MK_PRODUCER_WAIT)) return false;
-        if (!ring_throttle(r, a.err, DERR_MK_PRODUCER_WAIT)) return false;
         uint8_t* dst = r.stages + r.st * GV_UNIT_BYTES;
         const int row = (int)((long long)l * a.kv_rows_per_layer + (long long)gr * a.S_max + j * AK);
         mbar_arrive_expect_tx(&r.full[r.st], GV_UNIT_BYTES);
@@ -184,10 +183,7 @@ DEVI void attn_consume(GvRing& ring, const DecodeStepArgs& a, int l, const AttnS
                 }
             }
             __syncwarp();
-            if (lane == 0) {
-                __threadfence();
-                atomicAdd(cnt, 1u);
-            }
+            if (lane == 0) red_release_add(cnt, 1u);
             __syncwarp();
             return;
         }
@@ -386,9 +382,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
     uint64_t* full = reinterpret_cast<uint64_t*>(xs_raw + a.xs_bytes);
     __shared__ float rinv_s[16];
     __shared__ float rred_s[8][16];
-    __shared__ int last_s;
     __shared__ int s_len[16];  // cache lengths before this step (the new token's positions)
-    GvRing ring{smem, full, full + a.n_stages, a.n_stages, 0, 0u, a.inflight_units, 0};
+    GvRing ring{smem, full, full + a.n_stages, a.n_stages, 0, 0u, 0};
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const int B = a.B, D = a.D, Hd = a.H * a.d, Hkd = a.Hk * a.d, F = a.F;
@@ -486,8 +481,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
             e.k_cache = kc;
             e.v_cache = vc;
             const GvX X = token_rows(a.hw, D, ds_norm(a, nparts));
-            gv_consume<NB, EPI_QKV_ROPE, true>(ring, gv_work(nt_qkv, nku_D), X, Hd + 2 * Hkd, 0, rinv_s, e, a.ws,
-                                         a.max_pieces[0], &last_s, a.err, DERR_MK_CONSUMER_WAIT);
+            gv_consume<NB, EPI_QKV_ROPE>(ring, gv_work(nt_qkv, nku_D), X, Hd + 2 * Hkd, 0, rinv_s, e, a.ws,
+                                         a.max_pieces[0], a.err, DERR_MK_CONSUMER_WAIT);
             if (!barrier()) return;
         }
         // attention over the cache (the new token's K and V included)
@@ -504,8 +499,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
             e.ss_out = a.ss;
             e.ss_out_ld = a.ss_ld;
             const GvX X = token_rows(a.o, Hd, NormIn());
-            gv_consume<NB, EPI_RESID, true>(ring, gv_work(nt_D, nku_Hd), X, D, 0, rinv_s, e, a.ws, a.max_pieces[1],
-                                      &last_s, a.err, DERR_MK_CONSUMER_WAIT);
+            gv_consume<NB, EPI_RESID>(ring, gv_work(nt_D, nku_Hd), X, D, 0, rinv_s, e, a.ws, a.max_pieces[1],
+                                      a.err, DERR_MK_CONSUMER_WAIT);
             nparts = resid_parts;
             if (!barrier()) return;
         }
@@ -516,8 +511,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
             e.g_out = a.g;
             e.F = F;
             const GvX X = token_rows(a.hw, D, ds_norm(a, nparts));
-            gv_consume<NB, EPI_SWIGLU, true>(ring, gv_work(nt_F, nku_D), X, F, 0, rinv_s, e, a.ws, a.max_pieces[2],
-                                       &last_s, a.err, DERR_MK_CONSUMER_WAIT);
+            gv_consume<NB, EPI_SWIGLU>(ring, gv_work(nt_F, nku_D), X, F, 0, rinv_s, e, a.ws, a.max_pieces[2],
+                                       a.err, DERR_MK_CONSUMER_WAIT);
             if (!barrier()) return;
         }
         // w2 + residual; writes the next norm's input
@@ -531,8 +526,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
             e.ss_out = a.ss;
             e.ss_out_ld = a.ss_ld;
             const GvX X = token_rows(a.g, F, NormIn());
-            gv_consume<NB, EPI_RESID, true>(ring, gv_work(nt_D, nku_F), X, D, 0, rinv_s, e, a.ws, a.max_pieces[3],
-                                      &last_s, a.err, DERR_MK_CONSUMER_WAIT);
+            gv_consume<NB, EPI_RESID>(ring, gv_work(nt_D, nku_F), X, D, 0, rinv_s, e, a.ws, a.max_pieces[3],
+                                      a.err, DERR_MK_CONSUMER_WAIT);
             if (!barrier()) return;
         }
     }
@@ -548,8 +543,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
         e.seq_len = a.seq_len;
         e.advance = 1;
         const GvX X = token_rows(a.hw, D, ds_norm(a, nparts));
-        gv_consume<NB, EPI_LOGITS, true>(ring, gv_work(nt_V, nku_D), X, a.vocab, 0, rinv_s, e, a.ws, a.max_pieces[4],
-                                   &last_s, a.err, DERR_MK_CONSUMER_WAIT);
+        gv_consume<NB, EPI_LOGITS>(ring, gv_work(nt_V, nku_D), X, a.vocab, 0, rinv_s, e, a.ws, a.max_pieces[4],
+                                   a.err, DERR_MK_CONSUMER_WAIT);
     } else {
         // layer stack only: hand out the hidden states and advance the cache lengths
         const long long n4 = (long long)B * D / 4;

@@ -76,8 +76,7 @@ __global__ void __launch_bounds__(GV_THREADS, 2)
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + GV_STAGES * GV_UNIT_BYTES + GV_XS_BYTES);
     __shared__ float rinv_s[16];
     __shared__ float rred_s[8][16];
-    __shared__ int last_s;
-    GvRing ring{smem, full, full + GV_STAGES, GV_STAGES, 0, 0u, 0, 0};
+    GvRing ring{smem, full, full + GV_STAGES, GV_STAGES, 0, 0u, 0};
     const int warp = threadIdx.x >> 5;
     const GvWork w = gv_work(ntiles, nku);
 
@@ -115,8 +114,7 @@ __global__ void __launch_bounds__(GV_THREADS, 2)
     X.Kp = nku * GV_BK;
     X.xs = (long long)a.M * X.Kp * 2 <= GV_XS_BYTES ? xs : nullptr;
     gv_prologue(const_cast<__nv_bfloat16*>(X.xs), a.x, a.ldx, a.M, a.K, X.Kp, a.epi.norm, a.m0, rinv_s, rred_s);
-    gv_consume<NB, EPI, true>(ring, w, X, a.N, a.m0, rinv_s, a.epi, a.ws, max_pieces, &last_s, a.epi.err,
-                              DERR_GEMV_CONSUMER_WAIT);
+    gv_consume<NB, EPI>(ring, w, X, a.N, a.m0, rinv_s, a.epi, a.ws, max_pieces, a.epi.err, DERR_GEMV_CONSUMER_WAIT);
 }
 
 // fp32 kernel (CUDA cores): a warp owns a pair of logical rows, a CTA 8 pairs.
@@ -256,9 +254,9 @@ static cudaError_t launch_bf16_e(const GemvArgs<__nv_bfloat16>& a, cudaStream_t 
     }
     if (!a.tmw[0]) return cudaErrorInvalidValue;
     const GemvPlan p = gemv_plan(EPI, a.N, a.K, a.num_sms, 1);
-    if ((size_t)p.ntiles * p.max_pieces * GV_PIECE_FLOATS > a.ws.part_floats || p.ntiles > a.ws.tiles_cap)
+    if ((size_t)p.ntiles * p.max_pieces * GV_PIECE_FLOATS > a.ws.part_floats || p.ntiles > a.ws.tiles_cap ||
+        !a.ws.warp_cnt)
         return cudaErrorInvalidValue;
-    if (!a.ws.warp_cnt) return cudaErrorInvalidValue;
     const CUtensorMap& m0 = *a.tmw[0];
     const CUtensorMap& m1 = a.tmw[1] ? *a.tmw[1] : m0;
     const CUtensorMap& m2 = a.tmw[2] ? *a.tmw[2] : m0;

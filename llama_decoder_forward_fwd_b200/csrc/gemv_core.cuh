@@ -15,11 +15,11 @@
 // consume every unit with mma.sync m16n8k16 (weights as the A operand, token
 // rows as B), so no reduction between warps is needed. A row tile whose k range
 // is split over several CTAs leaves one partial per CTA, added in CTA order (so
-// results are deterministic) by one CTA whose warps then run the fused epilogue:
-// in a launch that may not have all CTAs resident, the CTA that completes the
-// tile (atomic counter, no waiting); in the cooperative fused decode step, the
-// tile's first CTA (which reaches the tile last, at the end of its range), each
-// of its warps waiting for the other CTAs' pieces of its own 16 rows.
+// results are deterministic) by the tile's first CTA, which reaches the tile
+// last (at the end of its range): each of its warps waits for the other CTAs'
+// pieces of its own 16 rows and runs the fused epilogue. The other CTAs publish
+// their pieces and move on. Both kernels that use this are launched
+// cooperatively, so every CTA is resident while the first ones wait.
 //
 // Fragment layout: lane (g = lane/4, t = lane%4) reads 16 contiguous bf16 of its
 // rows g and g+8 at k0 + 16t. Because a dot product does not depend on the order
@@ -70,23 +70,8 @@ struct GvRing {
     int n;
     int st;
     uint32_t ph;
-    int inflight;     // producer: most copies in flight (issued, not landed); 0 = up to n
     long long issued; // producer: copies issued so far
 };
-// Producer, before issuing a copy: with a limit on copies in flight, wait until
-// the copy issued `inflight` units ago has landed. Copies beyond the few that
-// keep HBM busy only lengthen the memory system's queues, and with them the
-// latency of every dependent load, atomic and fence of the consumers.
-DEVI bool ring_throttle(GvRing& r, uint32_t* err, uint32_t code) {
-    if (r.inflight <= 0 || r.inflight >= r.n || r.issued < r.inflight) return true;
-    int s = r.st - r.inflight;
-    uint32_t p = r.ph;
-    if (s < 0) {
-        s += r.n;
-        p ^= 1u;
-    }
-    return mbar_wait(&r.full[s], p, err, code);
-}
 DEVI void ring_next(GvRing& r) {
     if (++r.st == r.n) {
         r.st = 0;
@@ -130,7 +115,6 @@ DEVI bool gv_produce(GvRing& r, const GvWork& w, bool swiglu, const CUtensorMap*
     int tile = (int)(w.u0 / w.nku), kb = (int)(w.u0 % w.nku);  // tracked incrementally: no division in the loop
     for (long long u = w.u0; u < w.u1; ++u) {
         if (!mbar_wait(&r.empty[r.st], r.ph ^ 1u, err, code)) return false;
-        if (!ring_throttle(r, err, code)) return false;
         uint8_t* dst = r.stages + r.st * GV_UNIT_BYTES;
         const int kx = kb * GV_BK;
         mbar_arrive_expect_tx(&r.full[r.st], GV_UNIT_BYTES);
@@ -363,9 +347,9 @@ DEVI void gv_epilogue(int tile, const float (&c)[NB / 8][4], int N, int M, int m
 // tile reduction and the epilogues. A failed (timed-out) wait is recorded in
 // *err; the warp then stops waiting and runs the rest of its control flow on
 // whatever the stage holds, so every consumer warp still reaches every barrier.
-template <int NB, int EPI, bool OWNER = false>
+template <int NB, int EPI>
 DEVI bool gv_consume(GvRing& r, const GvWork& w, const GvX& X, int N, int m0, const float* rinv_s, const Epi& e,
-                     const GemvScratch& ws, int max_pieces, int* last_s, uint32_t* err, uint32_t code) {
+                     const GemvScratch& ws, int max_pieces, uint32_t* err, uint32_t code) {
     constexpr int NM = NB / 8;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t4 = lane & 3;
@@ -437,7 +421,7 @@ DEVI bool gv_consume(GvRing& r, const GvWork& w, const GvX& X, int N, int m0, co
         const long long cf = cta_of_unit(tu0, G, w.TU), cl = cta_of_unit(tu0 + w.nku - 1, G, w.TU);
         if (cf == cl) {
             gv_epilogue<NB, EPI>(tile, c, N, M, m0, rinv_s, e, ws, w.ntiles);
-        } else if (OWNER) {
+        } else {
             // Every CTA of the tile but the first publishes its piece, one warp's rows
             // at a time; the first CTA's warps wait for their rows' pieces.
             float* base = ws.part + (size_t)tile * max_pieces * GV_PIECE_FLOATS + (warp * 32 + lane) * 8;
@@ -449,10 +433,7 @@ DEVI bool gv_consume(GvRing& r, const GvWork& w, const GvX& X, int N, int m0, co
                 for (int n = 0; n < NM; ++n)
                     *reinterpret_cast<float4*>(mine + 4 * n) = make_float4(c[n][0], c[n][1], c[n][2], c[n][3]);
                 __syncwarp();
-                if (lane == 0) {
-                    __threadfence();
-                    atomicAdd(cnt, 1u);
-                }
+                if (lane == 0) red_release_add(cnt, 1u);
                 __syncwarp();
             } else {
                 if (lane == 0) {
@@ -474,38 +455,6 @@ DEVI bool gv_consume(GvRing& r, const GvWork& w, const GvX& X, int N, int m0, co
                 for (int n = 0; n < NM; ++n) t[n][0] = c[n][0], t[n][1] = c[n][1], t[n][2] = c[n][2], t[n][3] = c[n][3];
                 for (long long p = 1; p <= cl - cf; ++p) {
                     const float* src = base + (size_t)p * GV_PIECE_FLOATS;
-#pragma unroll
-                    for (int n = 0; n < NM; ++n) {
-                        const float4 v = __ldcg(reinterpret_cast<const float4*>(src + 4 * n));
-                        t[n][0] += v.x;
-                        t[n][1] += v.y;
-                        t[n][2] += v.z;
-                        t[n][3] += v.w;
-                    }
-                }
-                gv_epilogue<NB, EPI>(tile, t, N, M, m0, rinv_s, e, ws, w.ntiles);
-            }
-        } else {
-            float* base = ws.part + (size_t)tile * max_pieces * GV_PIECE_FLOATS;
-            float* mine = base + (size_t)(blockIdx.x - cf) * GV_PIECE_FLOATS + (warp * 32 + lane) * 8;
-#pragma unroll
-            for (int n = 0; n < NM; ++n)
-                *reinterpret_cast<float4*>(mine + 4 * n) = make_float4(c[n][0], c[n][1], c[n][2], c[n][3]);
-            __threadfence();
-            named_bar_sync(1, GV_CONSUMERS);
-            if (threadIdx.x == 0) {
-                const unsigned prev = atomicAdd(ws.tile_cnt + tile, 1u);
-                *last_s = prev == (unsigned)(cl - cf);
-                if (*last_s) ws.tile_cnt[tile] = 0u;
-            }
-            named_bar_sync(1, GV_CONSUMERS);
-            if (*last_s) {
-                __threadfence();
-                float t[NM][4];
-#pragma unroll
-                for (int n = 0; n < NM; ++n) t[n][0] = t[n][1] = t[n][2] = t[n][3] = 0.f;
-                for (long long p = 0; p <= cl - cf; ++p) {
-                    const float* src = base + (size_t)p * GV_PIECE_FLOATS + (warp * 32 + lane) * 8;
 #pragma unroll
                     for (int n = 0; n < NM; ++n) {
                         const float4 v = __ldcg(reinterpret_cast<const float4*>(src + 4 * n));

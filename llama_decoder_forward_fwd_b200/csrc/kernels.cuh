@@ -86,8 +86,7 @@ enum { TM_WQ, TM_WK, TM_WV, TM_WO, TM_W1, TM_W3, TM_W2, TM_W1G, TM_W3G, TM_PER_L
 struct GemvScratch {
     float* part = nullptr;                  // partial fragments of split tiles
     size_t part_floats = 0;
-    unsigned* tile_cnt = nullptr;           // [tiles_cap] k blocks finished per tile
-    int tiles_cap = 0;
+    int tiles_cap = 0;                      // row tiles the counters below cover
     unsigned long long* am_best = nullptr;  // [16] packed (logit, id) maxima
     unsigned* done_cnt = nullptr;           // [1] tiles finished (argmax)
     unsigned* warp_cnt = nullptr;           // [tiles_cap * 8] pieces published per (tile, warp)
@@ -178,8 +177,6 @@ struct DecodeStepArgs {
     float eps = 0.f, scale_log2 = 0.f;
     int has_head = 0;
     int n_stages = 0, xs_bytes = 0;  // shared memory: ring stages; token rows / query tile
-    int prefetch_units = 0;          // units the producer prefetches into L2 ahead of its loads
-    int inflight_units = 0;          // most units in flight per CTA (0: the whole ring)
     int max_pieces[5] = {1, 1, 1, 1, 1};  // split-tile slots of QKV, wo, w1/w3, w2, lm_head
     // inputs and outputs of the step
     const int32_t* tok = nullptr;  // [B] token ids (models with embedding and head)
