@@ -227,11 +227,87 @@ struct GvX {
     const __nv_bfloat16* xs; // [M][Kp] copy in shared memory, or nullptr
 };
 
+// Operands of a tile's epilogue that live in global memory: for the residual
+// epilogue the old h values and the next norm weight of this lane's rows, for the
+// QKV epilogue the RoPE cos/sin of its rows at each token's position. They are
+// loaded when the tile's first unit is consumed -- only the CTA that holds the
+// tile's first unit runs its epilogue -- so they have arrived by the tile's end
+// instead of adding dependent L2 round trips to the end of the kernel.
+template <int NB>
+struct GvEpiOps {
+    float a[NB / 8][2][2];  // [n][h][row g / g+8]: residual h, or RoPE cos
+    float b[NB / 8][2][2];  // RoPE sin
+    float w[2];             // next norm weight of rows g / g+8
+};
+
+template <int NB, int EPI>
+DEVI void gv_epi_prefetch(GvEpiOps<NB>& op, int tile, int N, int M, int m0, const Epi& e) {
+    if (EPI != EPI_RESID && EPI != EPI_QKV_ROPE) return;
+    constexpr int NM = NB / 8;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t4 = lane & 3;
+    int lr[2];
+    lr[0] = tile * GV_ROWS + warp * 16 + g;
+    lr[1] = lr[0] + 8;
+    if (EPI == EPI_RESID) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+            op.w[q] = lr[q] < N ? to_f<__nv_bfloat16>(reinterpret_cast<const __nv_bfloat16*>(e.wnext)[lr[q]]) : 0.f;
+    }
+#pragma unroll
+    for (int n = 0; n < NM; ++n)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int m = n * 8 + 2 * t4 + h;
+            const int mg = m0 + m;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                op.a[n][h][q] = 0.f;
+                op.b[n][h][q] = 0.f;
+                if (m >= M || lr[q] >= N) continue;
+                if (EPI == EPI_RESID) {
+                    op.a[n][h][q] = __ldcg(e.h + (long long)mg * e.D + lr[q]);
+                } else if ((g & 1) == 0 && lr[q] < (e.H + e.Hk) * e.d) {
+                    const int bq = mg / e.T;
+                    const int pos = e.pos0[bq] + (mg - bq * e.T);
+                    const long long ti = (long long)pos * (e.d >> 1) + ((lr[q] % e.d) >> 1);
+                    op.a[n][h][q] = e.rope_cos[ti];
+                    op.b[n][h][q] = e.rope_sin[ti];
+                }
+            }
+        }
+}
+
+// QKV epilogue for one (even, odd) column pair with its RoPE cos/sin given:
+// rotate q and k, write q, append k and v to the cache at the token's position
+// (as epi_qkv_pair).
+DEVI void gv_qkv_pair(const Epi& e, int m, int col, float v0, float v1, float cs, float sn) {
+    const int Hd = e.H * e.d, Hkd = e.Hk * e.d;
+    const int b = m / e.T;
+    const int pos = e.pos0[b] + (m - b * e.T);
+    if (col < Hd + Hkd) {
+        const float r0 = v0 * cs - v1 * sn;
+        const float r1 = v0 * sn + v1 * cs;
+        v0 = r0;
+        v1 = r1;
+    }
+    if (col < Hd) {
+        store2<__nv_bfloat16>(reinterpret_cast<__nv_bfloat16*>(e.q_out) + (long long)m * Hd + col, v0, v1);
+    } else {
+        int cc = col - Hd;
+        const bool isv = cc >= Hkd;
+        if (isv) cc -= Hkd;
+        const int kvh = cc / e.d, dd = cc - kvh * e.d;
+        __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(isv ? e.v_cache : e.k_cache);
+        store2<__nv_bfloat16>(base + ((long long)(b * e.Hk + kvh) * e.S_max + pos) * e.d + dd, v0, v1);
+    }
+}
+
 // Fused epilogue of one warp's 16 rows of a finished row tile (accumulators c,
-// before the RMSNorm scale).
+// before the RMSNorm scale; global operands in op).
 template <int NB, int EPI>
 DEVI void gv_epilogue(int tile, const float (&c)[NB / 8][4], int N, int M, int m0, const float* rinv_s, const Epi& e,
-                      const GemvScratch& ws, int ntiles) {
+                      const GemvScratch& ws, int ntiles, const GvEpiOps<NB>& op) {
     constexpr int NM = NB / 8;
     constexpr int TR = EPI == EPI_SWIGLU ? GV_ROWS / 2 : GV_ROWS;  // logical rows per tile
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -261,8 +337,8 @@ DEVI void gv_epilogue(int tile, const float (&c)[NB / 8][4], int N, int M, int m
                 const float p1 = __shfl_xor_sync(0xffffffffu, v1, 4);
                 if (m < M && (g & 1) == 0) {
                     const int mg = m0 + m;
-                    if (lr0 >= 0) epi_qkv_pair<__nv_bfloat16>(e, mg, lr0, v0, p0);
-                    if (lr1 >= 0) epi_qkv_pair<__nv_bfloat16>(e, mg, lr1, v1, p1);
+                    if (lr0 >= 0) gv_qkv_pair(e, mg, lr0, v0, p0, op.a[n][h][0], op.b[n][h][0]);
+                    if (lr1 >= 0) gv_qkv_pair(e, mg, lr1, v1, p1, op.a[n][h][1], op.b[n][h][1]);
                 }
                 continue;
             }
@@ -275,13 +351,19 @@ DEVI void gv_epilogue(int tile, const float (&c)[NB / 8][4], int N, int M, int m
                 if (lr0 >= 0)
                     reinterpret_cast<__nv_bfloat16*>(e.g_out)[(size_t)mg * e.F + lr0] = __float2bfloat16_rn(swiglu(v0, v1));
             } else if (EPI == EPI_RESID) {
+                // residual add and the next norm's input hw = h * w (as epi_resid1,
+                // with h and w from the prefetch)
                 float sq = 0.f;
                 if (lr0 >= 0) {
-                    const float hn = epi_resid1<__nv_bfloat16>(e, mg, lr0, v0);
+                    const float hn = op.a[n][h][0] + v0;
+                    e.h[(long long)mg * e.D + lr0] = hn;
+                    reinterpret_cast<__nv_bfloat16*>(e.hw_out)[(long long)mg * e.D + lr0] = __float2bfloat16_rn(hn * op.w[0]);
                     sq += hn * hn;
                 }
                 if (lr1 >= 0) {
-                    const float hn = epi_resid1<__nv_bfloat16>(e, mg, lr1, v1);
+                    const float hn = op.a[n][h][1] + v1;
+                    e.h[(long long)mg * e.D + lr1] = hn;
+                    reinterpret_cast<__nv_bfloat16*>(e.hw_out)[(long long)mg * e.D + lr1] = __float2bfloat16_rn(hn * op.w[1]);
                     sq += hn * hn;
                 }
                 ssum[n][h] = sq;
@@ -365,7 +447,10 @@ DEVI bool gv_consume(GvRing& r, const GvWork& w, const GvX& X, int N, int m0, co
     for (int n = 0; n < NM; ++n) c[n][0] = c[n][1] = c[n][2] = c[n][3] = 0.f;
     int ctile = (int)(w.u0 / w.nku), ckb = (int)(w.u0 % w.nku);
     const uint32_t xbase = X.xs ? smem_u32(X.xs) : 0u;
+    GvEpiOps<NB> ops;
     for (long long u = w.u0; u < w.u1; ++u) {
+        // this CTA holds the tile's first unit, so it runs the tile's epilogue
+        if (ckb == 0) gv_epi_prefetch<NB, EPI>(ops, ctile, N, M, m0, e);
         if (ok && !mbar_wait(&r.full[r.st], r.ph, err, code)) ok = false;
         const uint32_t sp = smem_u32(r.stages + r.st * GV_UNIT_BYTES);
         const int kx = ckb * GV_BK;
@@ -420,7 +505,7 @@ DEVI bool gv_consume(GvRing& r, const GvWork& w, const GvX& X, int N, int m0, co
         const long long tu0 = (long long)tile * w.nku;
         const long long cf = cta_of_unit(tu0, G, w.TU), cl = cta_of_unit(tu0 + w.nku - 1, G, w.TU);
         if (cf == cl) {
-            gv_epilogue<NB, EPI>(tile, c, N, M, m0, rinv_s, e, ws, w.ntiles);
+            gv_epilogue<NB, EPI>(tile, c, N, M, m0, rinv_s, e, ws, w.ntiles, ops);
         } else {
             // Every CTA of the tile but the first publishes its piece, one warp's rows
             // at a time; the first CTA's warps wait for their rows' pieces.
@@ -464,7 +549,7 @@ DEVI bool gv_consume(GvRing& r, const GvWork& w, const GvX& X, int N, int m0, co
                         t[n][3] += v.w;
                     }
                 }
-                gv_epilogue<NB, EPI>(tile, t, N, M, m0, rinv_s, e, ws, w.ntiles);
+                gv_epilogue<NB, EPI>(tile, t, N, M, m0, rinv_s, e, ws, w.ntiles, ops);
             }
         }
 #pragma unroll
