@@ -384,6 +384,131 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- the other workloads
+def run_workload(args):
+    """Prefill and decode throughput of a workload other than the headline one (one GPU).
+
+    Token workloads: a prefill of the prompt, then greedy decode steps (CUDA
+    graphs). Hidden-state workloads: the layer stack on N(0,1) hidden states, then
+    hidden-state decode steps. Pre-filled-cache workloads: N(0,1) keys and values
+    written straight into the cache at the seeded ragged lengths (drawn on the
+    device: timing only, parity is the tests'), then decode steps.
+    """
+    import torch
+
+    import llama_decoder_forward_fwd_b200 as L
+    import seeded_inputs as S
+
+    w = S.WORKLOADS[args.workload]
+    shape, B, T, G = w.shape, w.batch, w.prompt_len, w.decode_steps
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    glob, layers = S.make_weights(shape, w.seed, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    graph = w.input_kind != "hidden" and not args.no_graph
+    flags = (L.LLM_FLAG_CUDA_GRAPH if graph else 0) | (L.LLM_FLAG_FUSED_DECODE if args.fused else 0)
+    mt = B * T if T else B
+    model = L.Model(shape, glob, layers, max_batch=B, max_tokens=mt, flags=flags, stream=stream, device=dev)
+    D, Hk, d, Ln = shape.dim, shape.n_kv_heads, shape.head_dim, shape.n_layers
+    if w.input_kind == "kv_prefilled":
+        lens = S.make_kv_prefill(shape, w.seed, B, *w.kv_len_range, layers=[])[0].tolist()
+    else:
+        lens = [T] * B
+    tok0 = S.make_tokens(w.seed, B, max(T, 1), shape.vocab).to(dev)
+    hid = S.make_hidden(w.seed, B, T, D).to(dev) if w.input_kind == "hidden" else None
+    out_h = torch.empty_like(hid) if hid is not None else None
+    x1 = S.make_hidden(w.seed, B, 1, D, tag="decode")[:, 0].contiguous().to(dev) if hid is not None else None
+    o1 = torch.empty_like(x1) if x1 is not None else None
+    gen = torch.zeros(G + 1, B, dtype=torch.int32, device=dev)
+    gen[0] = S.make_tokens(w.seed, B, 1, shape.vocab, tag="decode0")[:, 0].to(dev)  # read by cache-only decode
+
+    def prefill():
+        L.llm_kv_cache_reset(model.h)
+        if w.input_kind == "tokens":
+            L.llm_prefill(model.h, tok0, gen[0])
+        elif w.input_kind == "hidden":
+            L.llm_prefill_hidden(model.h, hid, out_h)
+        else:
+            L.llm_kv_cache_set_lens(model.h, lens)
+
+    def decode():
+        for i in range(G):
+            if w.input_kind == "hidden":
+                L.llm_decode_step_hidden(model.h, x1, o1)
+            else:
+                L.llm_decode_step(model.h, gen[i], gen[i + 1])
+
+    if w.input_kind == "kv_prefilled":
+        kc, vc = model.kv_cache_tensors()
+        kc.normal_()
+        vc.normal_()
+        torch.cuda.synchronize(dev)
+    for _ in range(args.warmup):
+        prefill()
+        decode()
+    torch.cuda.synchronize(dev)
+    pre_ms, dec_ms = [], []
+    with ClockSampler(0) as clk:
+        for _ in range(args.steps):
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0.record(stream)
+            prefill()
+            e1.record(stream)
+            decode()
+            e2.record(stream)
+            torch.cuda.synchronize(dev)
+            pre_ms.append(e0.elapsed_time(e1))
+            dec_ms.append(e1.elapsed_time(e2))
+    L.llm_synchronize(model.h)
+    model.free()
+    # per-kernel decode time: a second pass with the library's CUDA-event timing
+    tm = L.Model(shape, model.glob, model.layers, max_batch=B, max_tokens=mt,
+                 flags=flags | L.LLM_FLAG_KERNEL_TIMING, stream=stream, device=dev)
+    model = tm
+    if w.input_kind == "kv_prefilled":
+        kc, vc = model.kv_cache_tensors()
+        kc.normal_()
+        vc.normal_()
+        torch.cuda.synchronize(dev)
+    for rep in range(2):  # the first pass captures the graphs
+        prefill()
+        L.llm_kernel_times(model.h, reset=True)
+        decode()
+        kt = L.llm_kernel_times(model.h, reset=True)
+    model.free()
+    # algorithmic work: every weight once per decode step, each sequence's cache once
+    head = shape.has_embed_and_head
+    S_mean = sum(lens) / B + G / 2
+    prefill_flops, _, kind_bytes, _ = work_model(shape, B, T, S_mean)
+    kernels = {k: {"ms_per_step": ms / G, "launches_per_step": n / G,
+                   "gbs": (kind_bytes[k] * n / G) / (ms / G) / 1e6 if k in kind_bytes and ms else None}
+               for k, (ms, n) in kt.items() if n}
+    lin_params = Ln * (D * (shape.n_heads + 2 * Hk) * d + shape.n_heads * d * D + 3 * D * shape.ffn_hidden)
+    esz = 2 if shape.dtype == "bf16" else 4
+    if not head:
+        prefill_flops -= 2 * B * D * shape.vocab
+    step_bytes = esz * (lin_params + (shape.vocab * D if head else 0)) + Ln * B * 2 * Hk * d * esz * S_mean
+    dec_s = statistics.median(dec_ms) / 1e3
+    line = {"impl": "ours", "workload": w.name, "metric": "decode tokens/s; % of measured HBM (and prefill % of bf16 peak)",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "dtype": shape.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "batch": B, "prompt_len": T, "decode_steps": G, "input": w.input_kind,
+                       "cache_lengths": [min(lens), max(lens)], "cuda_graph_decode": graph,
+                       "decode_kernel": "fused step" if args.fused else "layerwise"},
+            "decode": {"tok_s": B * G / dec_s, "ms_per_step": dec_s * 1e3 / G, "gbs": step_bytes * G / dec_s / 1e9,
+                       "frac_of_hbm": step_bytes * G / dec_s / 1e9 / peaks["hbm_gbs"], "bytes_per_step": step_bytes,
+                       "peak_gbs": peaks["hbm_gbs"], "peak_source": peak_src, "kernels": kernels},
+            "clocks": clk.summary()}
+    if w.input_kind != "kv_prefilled":
+        pre_s = statistics.median(pre_ms) / 1e3
+        line["prefill"] = {"tok_s": B * T / pre_s, "ms": pre_s * 1e3, "tflops": prefill_flops / pre_s / 1e12,
+                           "frac_of_bf16_peak": (prefill_flops / pre_s / 1e12 / peaks["bf16_tflops"]
+                                                 if shape.dtype == "bf16" else None)}
+    line["value"] = line["decode"]["tok_s"]
+    line["unit"] = "tokens/s"
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -397,7 +522,13 @@ def main():
     ap.add_argument("--fused", action="store_true",
                     help="decode each step as the fused single-launch kernel instead of one launch per "
                          "projection and attention")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="another workload of seeded_inputs.WORKLOADS: prefill and decode throughput on one GPU "
+                         "(the default is the headline benchmark)")
     args = ap.parse_args()
+    if args.workload != WORKLOAD and args.impl == "ours":
+        run_workload(args)
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

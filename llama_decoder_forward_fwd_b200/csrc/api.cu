@@ -705,11 +705,13 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
     MALLOC_OR_BAIL(m->am_counter, 64);
     {
         // Attention scratch: the largest split-KV plan any call can request
-        // (decode, and prefill of fp32 or non-128 head_dim models).
+        // (decode, and prefill of fp32 or non-128 head_dim models). The plan's
+        // size is not monotone in T (the split count fills the GPU per group), so
+        // every T is evaluated; a plan is a few integer operations.
         size_t pf = 0, cn = 0;
         const int Tmax = (m->bf16 && d == 128) ? 1 : (int)(Mx < (size_t)c.max_seq_len ? Mx : c.max_seq_len);
         for (int B = 1; B <= c.max_batch; ++B)
-            for (int T = 1; T <= Tmax && (size_t)B * T <= Mx; T = (T < 16 ? T + 1 : T * 2)) {
+            for (int T = 1; T <= Tmax && (size_t)B * T <= Mx; ++T) {
                 const AttnDecodePlan p = attn_decode_plan(B, T, H, Hk, d, c.max_seq_len, m->num_sms);
                 pf = p.part_floats > pf ? p.part_floats : pf;
                 cn = p.counters > cn ? p.counters : cn;
@@ -1197,7 +1199,8 @@ int llm_op_attention_decode(const void* q, const void* kcache, const void* vcach
     if (rc) return rc;
     if ((H / Hk) > 16) return fail(LLM_ERR_UNSUPPORTED, "more than 16 query heads per KV head");
     if (!workspace) return fail(LLM_ERR_NULL_PTR, "workspace is NULL");
-    const AttnDecodePlan p = attn_decode_plan(B, T, H, Hk, d, 1 << 30, num_sms_current());
+    // planned for keys up to the cache length; the workspace size (any length) covers it
+    const AttnDecodePlan p = attn_decode_plan(B, T, H, Hk, d, S_max, num_sms_current());
     const size_t part_bytes = (p.part_floats * 4 + 255) & ~size_t(255);
     if (workspace_bytes < part_bytes + p.counters * 4 || !aligned16(workspace))
         return fail(LLM_ERR_BAD_ARG, "workspace too small or misaligned");

@@ -6,6 +6,7 @@
 namespace lfw {
 
 constexpr int AD_WARPS = 4;
+constexpr int AD_KEYS_PER_CTA = 704;
 constexpr int AD_THREADS = AD_WARPS * 32;
 
 template <typename KT, int RMAX>
@@ -25,10 +26,16 @@ AttnDecodePlan attn_decode_plan(int B, int T, int H, int Hk, int d, int max_keys
     if (p.tq < 1) p.tq = 1;
     p.n_qchunks = (T + p.tq - 1) / p.tq;
     const int groups = B * Hk * p.n_qchunks;
-    // About 128 keys per CTA (one 32-key group per warp), at least one CTA per SM,
-    // at least 32 keys per split.
-    const int by_len = (max_keys + 127) / 128;
-    const int fill = (num_sms + groups - 1) / groups;
+    // The kernel's register use leaves room for two CTAs per SM. Split so that all
+    // CTAs are resident at once (about 1.7 per SM: one wave, no tail) unless that
+    // leaves a CTA more than AD_KEYS_PER_CTA keys, then split by length instead.
+    // Measured on B200 (Llama-3-8B heads): batch 1 over 2304 keys is fastest at
+    // 24-32 splits, batch 4 over ~2k keys at 8, batch 16 over 4k-8k keys at 12;
+    // fewer splits leave SMs idle, more pay each CTA's fixed cost (query staging,
+    // one load round trip, the partial write and the split merge) more often.
+    // Every split keeps at least 32 keys.
+    const int fill = (num_sms * 7 / 4) / groups;
+    const int by_len = (max_keys + AD_KEYS_PER_CTA - 1) / AD_KEYS_PER_CTA;
     const int cap = (max_keys + AD_GK - 1) / AD_GK;
     int ns = by_len > fill ? by_len : fill;
     if (ns > cap) ns = cap;
