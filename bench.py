@@ -61,6 +61,33 @@ def work_model(shape, B, T, S_decode_mean):
     return prefill_flops, w_bytes + kv_bytes, kinds_bytes, kinds_flops
 
 
+# ---------------------------------------------------------------- replicas
+# With N > 1 every rank runs its own replica of the whole workload on its own GPU;
+# the ranks meet only to line up the timed region and to take the slowest rank's
+# time. These helpers take the process group torch.distributed already holds
+# (nccl on GPUs, gloo in the CPU tests) and the device its tensors live on.
+def replica_barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def replica_max(x: float, world: int, device) -> float:
+    """The largest x over all ranks (every rank gets it)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world: int, steps: int, units_per_step: float, max_seconds: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return world * steps * units_per_step / max_seconds
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     def __init__(self, index: int):
@@ -218,7 +245,6 @@ def ncu_traffic(kind):
 # ---------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
-    import torch.distributed as dist
 
     import llama_decoder_forward_fwd_b200 as L
     import seeded_inputs as S
@@ -250,15 +276,10 @@ def run_ours(args, rank, world, local_rank):
             L.llm_decode_step(model.h, gen[i], gen[i + 1])
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        replica_barrier(world)
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replica_max(x, world, dev)
 
     for _ in range(args.warmup):
         one_step()
@@ -284,7 +305,7 @@ def run_ours(args, rank, world, local_rank):
     clocks = clk.summary()
     L.llm_synchronize(model.h)
     tokens_per_step = B * (T + G)
-    value = world * args.steps * tokens_per_step / total_s
+    value = replica_throughput(world, args.steps, tokens_per_step, total_s)
 
     S_mean = T + G / 2
     prefill_flops, decode_bytes, kbytes, kflops = work_model(shape, B, T, S_mean)
@@ -319,7 +340,7 @@ def run_ours(args, rank, world, local_rank):
         e_e[k].record(stream)
     torch.cuda.synchronize(dev)
     e2e_s = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)) / 1e3)
-    e2e = {"value": world * args.steps * tokens_per_step / e2e_s, "unit": "tokens/s",
+    e2e = {"value": replica_throughput(world, args.steps, tokens_per_step, e2e_s), "unit": "tokens/s",
            "h2d_bytes_per_step": host_prompt.numel() * 4, "d2h_bytes_per_step": host_out.numel() * 4}
 
     # ---- per-kernel CUDA-event timing of one step (roofline of the dominant kernel) ----
