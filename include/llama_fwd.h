@@ -88,7 +88,8 @@ extern "C" {
  * Model hyper-parameters: the params.json fields of "Building llama3 from
  * scratch" (dim, n_layers, n_heads, n_kv_heads, vocab_size, norm_eps, rope_theta),
  * plus the FFN hidden size given explicitly and the capacity limits.
- *   head_dim       must equal dim / n_heads; n_heads % n_kv_heads == 0.
+ *   head_dim       must equal dim / n_heads; n_heads % n_kv_heads == 0 (any
+ *                  group size: multi-head, grouped-query, multi-query).
  *   max_seq_len    KV-cache positions per sequence.
  *   max_batch      sequences (B) per call.
  *   max_tokens     B*T per prefill call (0 means max_batch * max_seq_len).
@@ -256,7 +257,8 @@ int llm_op_gemv_bf16(const void* x, const void* W, float* y, int M, int N, int K
  * Scale 1/sqrt(d); query head h reads KV head h / (H/Hk).
  * llm_op_attention_prefill is the flash (tensor-core) kernel: dtype LLM_BF16,
  * d == 128. llm_op_attention_decode is the split-KV kernel: any dtype,
- * d <= 128 with d % 8 == 0, H/Hk*T <= 16; it needs a device scratch buffer of
+ * d <= 128 with d % 8 == 0, any T and any H/Hk (multi-query included); it
+ * splits the keys by the cache length S_max and needs a device scratch buffer of
  * llm_op_attention_decode_workspace(...) bytes (16-byte aligned, contents
  * arbitrary; the kernel leaves it ready for the next call, so calls sharing one
  * buffer must not overlap in time).

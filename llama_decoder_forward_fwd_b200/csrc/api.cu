@@ -227,7 +227,6 @@ int validate_config(const llm_config* c) {
     if (c->dim % 8 != 0 || c->ffn_hidden % 8 != 0) return fail(LLM_ERR_BAD_CONFIG, "dim and ffn_hidden must be multiples of 8");
     if (c->dtype != LLM_F32 && c->dtype != LLM_BF16) return fail(LLM_ERR_BAD_CONFIG, "dtype must be LLM_F32 or LLM_BF16");
     if (c->has_embed_and_head && c->vocab <= 0) return fail(LLM_ERR_BAD_CONFIG, "vocab must be positive");
-    if (c->n_heads / c->n_kv_heads > 16) return fail(LLM_ERR_BAD_CONFIG, "more than 16 query heads per KV head");
     if (c->max_batch > 16) return fail(LLM_ERR_BAD_CONFIG, "max_batch > 16");
     if (c->dtype == LLM_BF16 && ((c->n_heads * c->head_dim) % 128 != 0 || (c->n_kv_heads * c->head_dim) % 128 != 0))
         return fail(LLM_ERR_BAD_CONFIG, "bf16 models need n_heads*head_dim and n_kv_heads*head_dim multiples of 128");
@@ -384,7 +383,7 @@ int run_layers(llm_model* m, int B, int T, int max_keys) {
             a.d = d;
             a.S_max = c.max_seq_len;
             a.n_splits = p.n_splits;
-            a.tq = p.tq;
+            a.rows = p.rows;
             a.n_qchunks = p.n_qchunks;
             a.ws_part = m->attn_ws;
             a.ws_count = m->attn_cnt;
@@ -1197,7 +1196,6 @@ int llm_op_attention_decode(const void* q, const void* kcache, const void* vcach
                             size_t workspace_bytes, void* stream) {
     int rc = attn_common_check(q, kcache, vcache, pos0, out, B, T, H, Hk, d, S_max, dtype);
     if (rc) return rc;
-    if ((H / Hk) > 16) return fail(LLM_ERR_UNSUPPORTED, "more than 16 query heads per KV head");
     if (!workspace) return fail(LLM_ERR_NULL_PTR, "workspace is NULL");
     // planned for keys up to the cache length; the workspace size (any length) covers it
     const AttnDecodePlan p = attn_decode_plan(B, T, H, Hk, d, S_max, num_sms_current());
@@ -1218,7 +1216,7 @@ int llm_op_attention_decode(const void* q, const void* kcache, const void* vcach
     a.d = d;
     a.S_max = S_max;
     a.n_splits = p.n_splits;
-    a.tq = p.tq;
+    a.rows = p.rows;
     a.n_qchunks = p.n_qchunks;
     a.ws_part = reinterpret_cast<float*>(workspace);
     a.ws_count = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(workspace) + part_bytes);

@@ -6,10 +6,11 @@
 // "KV cache" on the llama3.np page): query head h at position p attends to keys
 // 0..p of KV head h / G with scores q.k / sqrt(d) and a softmax.
 //
-// A work item is one (sequence, KV head, chunk of query tokens) and one
-// contiguous slice ("split") of the keys; its rows are the G query heads of the
-// KV head for each query token, so each key and value row is read once for the
-// whole group. Each of the NW warps takes 32-key groups of the split. Lane j
+// A work item is one (sequence, KV head, chunk of query rows) and one
+// contiguous slice ("split") of the keys. The rows of a KV head are its G query
+// heads at each query token, flattened as t*G + h; a chunk holds up to 16 of
+// them (whole tokens when G <= 16, part of one token's heads when G > 16), so
+// each key and value row is read once for all the rows of a chunk. Each of the NW warps takes 32-key groups of the split. Lane j
 // loads the whole key row j into registers and the value slice (dims 4l..4l+3)
 // of all 32 keys, every load issued before the first use, so a group costs one
 // memory round trip. Lane j scores key j for every row against the query rows,
@@ -80,7 +81,7 @@ DEVI void attn_split_item(const AttnDecodeArgs& a, int split, int b, int kvh, in
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.H / a.Hk, d = a.d;
-    const int R = a.tq * G;
+    const int R = a.rows;  // rows r of this item: (token, head) row0 + r, flattened as t*G + h
     const int HD = a.H * d;
     const int nch = d / EPC;
     const KT* q = reinterpret_cast<const KT*>(a.q);
@@ -89,8 +90,8 @@ DEVI void attn_split_item(const AttnDecodeArgs& a, int split, int b, int kvh, in
     const KT* vc = reinterpret_cast<const KT*>(a.vc) + head_off;
 
     const int p0 = a.pos0[b];
-    const int t_first = qc * a.tq;
-    const int t_last = min(a.T - 1, t_first + a.tq - 1);
+    const int row0 = qc * R;
+    const int t_last = min(a.T - 1, (row0 + R - 1) / G);
     // keys [0, limit) are visible to some row; never read past the cache
     const int limit = min(p0 + t_last + 1, a.S_max);
     int chunk = (limit + a.n_splits - 1) / a.n_splits;
@@ -120,16 +121,16 @@ DEVI void attn_split_item(const AttnDecodeArgs& a, int split, int b, int kvh, in
     for (int idx = threadIdx.x; idx < RMAX * (AD_DMAX / 4); idx += NT) {
         const int r = idx / (AD_DMAX / 4), dd = (idx % (AD_DMAX / 4)) * 4;
         float v[4] = {0.f, 0.f, 0.f, 0.f};
-        const int t = t_first + r / G;
+        const int t = (row0 + r) / G, hq = (row0 + r) % G;
         if (r < R && t < a.T && dd < d)
-            to4(__ldcg(reinterpret_cast<const V4*>(q + (long long)(b * a.T + t) * HD + (kvh * G + r % G) * d + dd)), v);
+            to4(__ldcg(reinterpret_cast<const V4*>(q + (long long)(b * a.T + t) * HD + (kvh * G + hq) * d + dd)), v);
         *reinterpret_cast<float4*>(&qs[r][dd]) =
             make_float4(v[0] * a.scale_log2, v[1] * a.scale_log2, v[2] * a.scale_log2, v[3] * a.scale_log2);
     }
     int plim[RMAX];  // last visible key of each row (-1: no row)
 #pragma unroll
     for (int r = 0; r < RMAX; ++r) {
-        const int t = t_first + r / G;
+        const int t = (row0 + r) / G;
         plim[r] = (r < R && t < a.T) ? p0 + t : -1;
     }
     named_bar_sync(1, NT);
@@ -297,9 +298,9 @@ DEVI void attn_split_item(const AttnDecodeArgs& a, int split, int b, int kvh, in
             acc.z += w * v.z;
             acc.w += w * v.w;
         }
-        const int t = t_first + r / G;
+        const int t = (row0 + r) / G, hq = (row0 + r) % G;
         if (t < a.T) {
-            KT* dst = out + (long long)(b * a.T + t) * HD + (kvh * G + r % G) * d + d4;
+            KT* dst = out + (long long)(b * a.T + t) * HD + (kvh * G + hq) * d + d4;
             dst[0] = from_f<KT>(acc.x);
             dst[1] = from_f<KT>(acc.y);
             dst[2] = from_f<KT>(acc.z);

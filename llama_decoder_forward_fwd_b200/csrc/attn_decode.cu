@@ -22,9 +22,12 @@ __global__ void __launch_bounds__(AD_THREADS) attn_decode_kernel(const AttnDecod
 AttnDecodePlan attn_decode_plan(int B, int T, int H, int Hk, int d, int max_keys, int num_sms) {
     AttnDecodePlan p;
     const int G = H / Hk;
-    p.tq = G >= 16 ? 1 : (16 / G < T ? 16 / G : T);
-    if (p.tq < 1) p.tq = 1;
-    p.n_qchunks = (T + p.tq - 1) / p.tq;
+    // Rows of a work item: the G query heads of 16/G whole tokens when G <= 16,
+    // else 16 of the G heads of one token (multi-query models).
+    int tq = G >= 16 ? 1 : (16 / G < T ? 16 / G : T);
+    if (tq < 1) tq = 1;
+    p.rows = G >= 16 ? 16 : tq * G;
+    p.n_qchunks = (int)(((long long)T * G + p.rows - 1) / p.rows);
     const int groups = B * Hk * p.n_qchunks;
     // The kernel's register use leaves room for two CTAs per SM. Split so that all
     // CTAs are resident at once (about 1.7 per SM: one wave, no tail) unless that
@@ -42,7 +45,7 @@ AttnDecodePlan attn_decode_plan(int B, int T, int H, int Hk, int d, int max_keys
     if (ns > AD_MAX_SPLITS) ns = AD_MAX_SPLITS;
     if (ns < 1) ns = 1;
     p.n_splits = ns;
-    p.part_floats = (size_t)groups * p.tq * G * ns * (d + 4);
+    p.part_floats = (size_t)groups * p.rows * ns * (d + 4);
     p.counters = groups;
     return p;
 }
@@ -54,9 +57,8 @@ static cudaError_t launch_one(const AttnDecodeArgs& a, cudaStream_t s, bool pdl)
 }
 
 cudaError_t launch_attn_decode(const AttnDecodeArgs& a, bool bf16, cudaStream_t s, bool pdl) {
-    const int G = a.H / a.Hk;
-    const int R = a.tq * G;
-    if (a.H % a.Hk != 0 || R > 16 || a.d > AD_DMAX || a.d % 8 != 0 || a.n_splits > AD_MAX_SPLITS)
+    const int R = a.rows;
+    if (a.H % a.Hk != 0 || R < 1 || R > 16 || a.d > AD_DMAX || a.d % 8 != 0 || a.n_splits > AD_MAX_SPLITS)
         return cudaErrorInvalidValue;
     if (bf16) {
         if (R <= 4) return launch_one<__nv_bfloat16, 4>(a, s, pdl);

@@ -60,8 +60,7 @@ extern "C" int llm_op_attention_decode_static(const void* q, const void* kcache,
                                               const int32_t* pos0, void* out, int B, int T, int H, int Hk, int d,
                                               int S_max, int dtype, void* stream) {
     if (!q || !kcache || !vcache || !pos0 || !out) return lfw::set_error(LLM_ERR_NULL_PTR, "NULL operand");
-    if (B < 1 || T < 1 || H < 1 || Hk < 1 || H % Hk != 0 || S_max < 1 || d < 8 || d % 8 != 0 || d > 128 ||
-        H / Hk > 16)
+    if (B < 1 || T < 1 || H < 1 || Hk < 1 || H % Hk != 0 || S_max < 1 || d < 8 || d % 8 != 0 || d > 128)
         return lfw::set_error(LLM_ERR_BAD_ARG, "bad attention shape");
     if (dtype != LLM_F32 && dtype != LLM_BF16) return lfw::set_error(LLM_ERR_BAD_ARG, "bad dtype");
     for (const void* p : {q, kcache, vcache, (const void*)out})
@@ -88,7 +87,7 @@ extern "C" int llm_op_attention_decode_static(const void* q, const void* kcache,
     a.d = d;
     a.S_max = S_max;
     a.n_splits = plan.n_splits;
-    a.tq = plan.tq;
+    a.rows = plan.rows;
     a.n_qchunks = plan.n_qchunks;
     a.ws_part = reinterpret_cast<float*>(base);
     a.ws_count = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(base) + kScratchPartBytes);

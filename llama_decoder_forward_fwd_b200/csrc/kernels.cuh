@@ -157,14 +157,15 @@ struct AttnDecodeArgs {
     void* out = nullptr;       // [B*T][H*d]
     const int32_t* pos0 = nullptr;
     int B = 0, T = 0, H = 0, Hk = 0, d = 0, S_max = 0;
-    int n_splits = 1, tq = 1, n_qchunks = 1;
+    // a work item: `rows` consecutive (token, head-in-group) rows r = t*G + h of one KV head
+    int n_splits = 1, rows = 1, n_qchunks = 1;
     float* ws_part = nullptr;       // split partials (m, l, o[d])
     unsigned* ws_count = nullptr;   // [B*Hk*n_qchunks], zero between launches
     float scale_log2 = 0.f;
     uint32_t* err = nullptr;
 };
 struct AttnDecodePlan {
-    int n_splits, tq, n_qchunks;
+    int n_splits, rows, n_qchunks;
     size_t part_floats, counters;
 };
 AttnDecodePlan attn_decode_plan(int B, int T, int H, int Hk, int d, int max_keys, int num_sms);

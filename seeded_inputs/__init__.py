@@ -98,6 +98,13 @@ WORKLOADS: Dict[str, Workload] = {
         shape=_LLAMA3_8B.replace(max_seq_len=8192 + 128),
         batch=16, prompt_len=0, decode_steps=128, input_kind="kv_prefilled",
         kv_len_range=(4096, 8192)),
+    # Long-context single-sequence decode: the cache pre-filled to 8064 positions,
+    # 128 greedy steps up to the 8192-position Llama-3 context.
+    "llama3-8b-bf16-b1-kv8k-g128": Workload(
+        name="llama3-8b-bf16-b1-kv8k-g128",
+        shape=_LLAMA3_8B.replace(max_seq_len=8192),
+        batch=1, prompt_len=0, decode_steps=128, input_kind="kv_prefilled",
+        kv_len_range=(8064, 8064)),
     # Llama-2-7B-shaped multi-head (no GQA) model, batch 8.
     "llama2-7b-mha-bf16-b8-p1024-g256": Workload(
         name="llama2-7b-mha-bf16-b8-p1024-g256",

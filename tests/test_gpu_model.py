@@ -121,6 +121,44 @@ def test_llama2_mha_shape_two_layers(lib):
     _run_tokens_case(shape, seed=79, B=3, T=77, steps=4)
 
 
+def test_multi_query_llama3_layer_shape_two_layers(lib):
+    """One KV head for all 32 query heads (MQA, G = 32): the prefill runs the flash
+    kernel with 32 heads per KV head, decode splits each token's heads into two
+    16-row work items."""
+    shape = S.WORKLOADS["llama3-8b-bf16-b1-p2048-g256"].shape.replace(n_layers=2, n_kv_heads=1, max_seq_len=256)
+    _run_tokens_case(shape, seed=80, B=2, T=40, steps=4)
+
+
+def test_multi_query_f32_greedy_stream_and_logits(lib):
+    """fp32 MQA model (32 query heads of 16 dims, one KV head): the decode kernel
+    also runs the prefill, with (token, head) rows chunked 16 at a time; the same
+    greedy stream as the oracle and logits within 1e-4."""
+    s = S.ModelShape(dim=512, n_layers=2, n_heads=32, n_kv_heads=1, head_dim=16, ffn_hidden=1024, vocab=512,
+                     max_seq_len=64, norm_eps=1e-5, rope_theta=10000.0, dtype="f32", tie_embeddings=False)
+    T, steps = 9, 12
+    model, orc = build_pair(s, 81, batch=1, max_tokens=T)
+    prompt = S.make_tokens(81, 1, T, s.vocab)
+    nxt = torch.empty(1, dtype=torch.int32, device=DEV)
+    logits = torch.empty(1, s.vocab, device=DEV)
+    L.llm_prefill(model.h, prompt.to(DEV), nxt, logits)
+    L.llm_synchronize(model.h)
+    o_taps = []
+    o_next, o_logits = orc.prefill(prompt.numpy(), o_taps)
+    check_taps(gpu_taps(model, T), o_taps, tol=1e-5, what="prefill")
+    for step in range(steps + 1):
+        g = logits.cpu().numpy()
+        err = np.abs(g - o_logits).max() / np.abs(o_logits).max()
+        assert err <= F32_LOGIT_REL, f"step {step}: logits rel err {err:.2e}"
+        assert int(nxt[0]) == int(o_next[0]), f"step {step}: token {int(nxt[0])} vs {int(o_next[0])}"
+        if step == steps:
+            break
+        cur = nxt.clone()
+        L.llm_decode_step(model.h, cur, nxt, logits)
+        L.llm_synchronize(model.h)
+        o_next, o_logits = orc.decode(o_next)
+    model.free()
+
+
 def test_batched_decode_over_prefilled_ragged_caches(lib):
     """Llama-3-8B shape, batch 16, caches pre-filled with N(0,1) to ragged lengths."""
     w = S.WORKLOADS["llama3-8b-bf16-b16-kv4k8k-g128"]
@@ -143,6 +181,30 @@ def test_batched_decode_over_prefilled_ragged_caches(lib):
         checked += check_argmax(nxt.cpu().numpy(), o_logits)
     assert L.llm_kv_cache_get_lens(model.h, B) == [int(x) + 4 for x in lens]
     assert checked >= 4 * B // 2
+    model.free()
+
+
+def test_long_context_decode_up_to_the_8192_context(lib):
+    """Batch-1 decode against a cache of 8064 positions (two Llama-3-8B layers):
+    many 32-key groups per attention warp and the longest cache the context allows."""
+    w = S.WORKLOADS["llama3-8b-bf16-b1-kv8k-g128"]
+    shape = w.shape.replace(n_layers=2)
+    model, orc = build_pair(shape, w.seed, batch=1, max_tokens=1, flags=L.LLM_FLAG_CUDA_GRAPH)
+    lens, caches = S.make_kv_prefill(shape, w.seed, 1, *w.kv_len_range)
+    install_prefilled_cache(model, orc, lens.numpy(), caches)
+    del caches
+    tok = S.make_tokens(w.seed, 1, 1, shape.vocab, tag="decode0")[:, 0].numpy()
+    nxt = torch.empty(1, dtype=torch.int32, device=DEV)
+    logits = torch.empty(1, shape.vocab, device=DEV)
+    for step in range(3):
+        L.llm_decode_step(model.h, torch.as_tensor(tok, dtype=torch.int32).to(DEV), nxt, logits)
+        L.llm_synchronize(model.h)
+        o_taps = []
+        tok, o_logits = orc.decode(tok, o_taps)
+        check_taps(gpu_taps(model, 1), [t.reshape(1, -1) for t in o_taps], what=f"step {step}")
+        check_argmax(nxt.cpu().numpy(), o_logits)
+        assert rel_l2(logits.cpu().numpy(), o_logits) <= BF16_REL_L2
+    assert L.llm_kv_cache_get_lens(model.h, 1) == [int(lens[0]) + 3]
     model.free()
 
 

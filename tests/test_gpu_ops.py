@@ -77,6 +77,8 @@ ATTN_CASES = [
     (2, 130, 8, 2, [0, 64]),
     (1, 300, 32, 8, [0]),
     (2, 64, 4, 4, [3, 0]),
+    (1, 20, 32, 1, [0]),       # multi-query: 32 query heads share one KV head
+    (2, 9, 24, 1, [3, 0]),
 ]
 
 
@@ -97,7 +99,10 @@ def test_flash_attention_prefill_matches_oracle(lib, B, T, H, Hk, pos0):
 @pytest.mark.parametrize("dtype,d,tol", [(torch.bfloat16, 128, 6e-3), (torch.float32, 48, 2e-5),
                                          (torch.float32, 128, 2e-5)])
 @pytest.mark.parametrize("B,T,H,Hk,pos0", [(1, 1, 32, 8, [0]), (3, 1, 32, 8, [0, 37, 700]),
-                                           (2, 4, 8, 2, [9, 0]), (1, 8, 6, 6, [0]), (2, 3, 12, 3, [100, 1])])
+                                           (2, 4, 8, 2, [9, 0]), (1, 8, 6, 6, [0]), (2, 3, 12, 3, [100, 1]),
+                                           # multi-query (G = 32, 24): a work item takes 16 of a
+                                           # token's query heads; with G = 24 chunks straddle tokens
+                                           (1, 1, 32, 1, [500]), (2, 3, 32, 1, [100, 7]), (1, 2, 24, 1, [50])])
 def test_split_kv_attention_matches_oracle(lib, dtype, d, tol, B, T, H, Hk, pos0):
     import llama_decoder_forward_fwd_b200 as L
     S = 1024
