@@ -1,8 +1,11 @@
 """Whole-model parity: the CUDA path through the C ABI against the fp64 oracle (GPU).
 
-All five workload shapes are covered; the Llama-3-8B and Llama-2-7B shapes run
-with 2 layers here (the layer is identical at any depth; full-depth runs are
-in test_gpu_fullsize.py). Decode steps feed both sides the oracle's own greedy
+Every workload shape is covered (the tiny fp32 model, one Llama-3-8B layer on
+hidden states, the Llama-3-8B shape at batch 1 and batch 16 over ragged caches,
+long-context decode at 8064+ positions, the Llama-2-7B MHA shape), plus
+multi-query variants; the Llama-3-8B and Llama-2-7B shapes run with 2 layers
+here (the layer is identical at any depth; full-depth runs are in
+test_gpu_fullsize.py). Decode steps feed both sides the oracle's own greedy
 token, so no value computed on the GPU is ever an oracle input.
 """
 import numpy as np
