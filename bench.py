@@ -8,6 +8,7 @@ of the Llama-3-8B architecture (32 layers, dim 4096, 32/8 heads, FFN 14336,
 vocab 128256). Inputs are resident in HBM when the timed region starts.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --workload NAME [--steps K] [--warmup W] [--fused]   # another seeded workload
 
 For N > 1 run under torch.distributed.run: every rank runs an independent
 replica on its own GPU (the decoder has no exchange step), times are the max
@@ -547,8 +548,11 @@ def main():
                     help="another workload of seeded_inputs.WORKLOADS: prefill and decode throughput on one GPU "
                          "(the default is the headline benchmark)")
     args = ap.parse_args()
-    if args.workload != WORKLOAD and args.impl == "ours":
-        run_workload(args)
+    if args.workload != WORKLOAD:
+        if args.impl == "ours":
+            run_workload(args)
+        elif int(os.environ.get("RANK", "0")) == 0:
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm times the headline workload only"}))
         return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -27,7 +27,6 @@ the error that rounding policy alone produces. (The GPU's distance to the
 rounding-policy oracle is printed but not bounded: the two round from slightly
 different fp32 intermediates, so their rounding errors are largely independent.)
 """
-import numpy as np
 import pytest
 import torch
 

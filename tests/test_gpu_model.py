@@ -13,9 +13,8 @@ import pytest
 import torch
 
 import llama_decoder_forward_fwd_b200 as L
-import oracle as O
 import seeded_inputs as S
-from model_util import (ARGMAX_MARGIN, BF16_REL_L2, F32_LOGIT_REL, build_pair, check_argmax, check_taps,
+from model_util import (BF16_REL_L2, F32_LOGIT_REL, build_pair, check_argmax, check_taps,
                         gpu_taps, install_prefilled_cache, rel_l2)
 
 pytestmark = pytest.mark.gpu
