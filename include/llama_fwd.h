@@ -68,9 +68,10 @@ extern "C" {
 #define LLM_FLAG_FUSED_DECODE  16 /* run each bf16 decode step as one persistent launch (the
                                     whole model: every layer's projections and attention and the
                                     lm_head, separated by grid barriers) instead of one launch per
-                                    projection and attention; needs head_dim 128 and a dim that
-                                    is a multiple of 256, and is not used with
-                                    LLM_FLAG_DEBUG_TAPS */
+                                    projection and attention; needs head_dim 128, a dim that is
+                                    a multiple of 256 and at most 16 query heads per KV head,
+                                    and is not used with LLM_FLAG_DEBUG_TAPS; other models
+                                    decode with the per-kernel path */
 
 /* ---- kernel kinds reported by llm_kernel_times ------------------------- */
 #define LLM_K_EMBED    0   /* embedding lookup / hidden-state load */
@@ -88,10 +89,13 @@ extern "C" {
  * Model hyper-parameters: the params.json fields of "Building llama3 from
  * scratch" (dim, n_layers, n_heads, n_kv_heads, vocab_size, norm_eps, rope_theta),
  * plus the FFN hidden size given explicitly and the capacity limits.
- *   head_dim       must equal dim / n_heads; n_heads % n_kv_heads == 0 (any
- *                  group size: multi-head, grouped-query, multi-query).
+ *   head_dim       must equal dim / n_heads, be a multiple of 8 and at most
+ *                  128; n_heads % n_kv_heads == 0 (any group size: multi-head,
+ *                  grouped-query, multi-query).
+ *   dim, ffn_hidden multiples of 8; for LLM_BF16 also n_heads*head_dim and
+ *                  n_kv_heads*head_dim multiples of 128.
  *   max_seq_len    KV-cache positions per sequence.
- *   max_batch      sequences (B) per call.
+ *   max_batch      sequences (B) per call, at most 16.
  *   max_tokens     B*T per prefill call (0 means max_batch * max_seq_len).
  *   dtype          LLM_F32 or LLM_BF16 (type of every weight buffer).
  *   tie_embeddings lm_head reuses tok_emb (weights.out ignored).
