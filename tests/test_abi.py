@@ -86,3 +86,19 @@ def test_op_shape_checks_are_host_side(lib):
     assert lib.llm_op_gemv_bf16(p, p, p, 17, 16, 64, p, 1 << 20, None) == L.LLM_ERR_BAD_ARG  # M > 16
     assert lib.llm_op_attention_decode_workspace(1, 1, 32, 8, 128) > 0
     assert lib.llm_op_attention_decode_workspace(1, 1, 30, 8, 128) == 0             # H % Hk
+
+
+@pytest.mark.parametrize("B,T,H,Hk,d,items,rows", [
+    (1, 1, 32, 8, 128, 8, 4),    # GQA decode: each of 8 KV heads has one item of its 4 query heads
+    (1, 5, 12, 3, 64, 6, 16),    # G = 4, T = 5: 4 whole tokens (16 rows) + 1 token, per KV head
+    (1, 1, 32, 1, 128, 2, 16),   # multi-query decode: 32 rows of one token -> 2 items of 16
+    (1, 2, 24, 1, 128, 3, 16),   # G = 24, T = 2: 48 rows -> 3 items, the second straddles the tokens
+    (2, 3, 32, 1, 48, 12, 16),   # 96 rows per sequence -> 6 items, 2 sequences
+])
+def test_split_kv_workspace_follows_the_16_row_work_items(lib, B, T, H, Hk, d, items, rows):
+    """The workspace is sized for the plan's work items (sequence, KV head, up to 16
+    (token, head) rows) at the largest split count, 64: per item, split and row slot
+    one record (m, l, 2 pad, o[d]) of floats, then one merge counter per item."""
+    part = items * rows * 64 * (d + 4) * 4
+    expect = ((part + 255) & ~255) + items * 4
+    assert lib.llm_op_attention_decode_workspace(B, T, H, Hk, d) == expect
