@@ -29,6 +29,9 @@ MUTATIONS = {
     "ffn norm dropped": ('x = self._norm_in(h, w["ffn_norm"])', 'x = h * w["ffn_norm"]'),
     "attention residual dropped": ('h = h + out @ w["wo"].T', 'h = out @ w["wo"].T'),
     "final norm dropped": ('x = self._norm_in(h[:, -1, :], f64(self.glob["norm"]))', "x = h[:, -1, :]"),
+    "bf16 rounding keeps 9 bits": ("return np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)",
+                                   "return np.ldexp(np.rint(np.ldexp(m, 9)), e - 9)"),
+    "bf16 rounding truncates": ("np.rint(np.ldexp(m, 8))", "np.trunc(np.ldexp(m, 8))"),
     "argmax ties to the highest index": ("return np.argmax(logits, axis=-1)",
                                          "return logits.shape[-1] - 1 - np.argmax(logits[..., ::-1], axis=-1)"),
 }
