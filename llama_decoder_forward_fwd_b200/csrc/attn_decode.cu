@@ -30,7 +30,7 @@ AttnDecodePlan attn_decode_plan(int B, int T, int H, int Hk, int d, int max_keys
     p.n_qchunks = (int)(((long long)T * G + p.rows - 1) / p.rows);
     const int groups = B * Hk * p.n_qchunks;
     // The kernel's register use leaves room for two CTAs per SM. Split so that all
-    // CTAs are resident at once (about 1.7 per SM: one wave, no tail) unless that
+    // CTAs are resident at once (1.75 per SM: one wave, no tail) unless that
     // leaves a CTA more than AD_KEYS_PER_CTA keys, then split by length instead.
     // Measured on B200 (Llama-3-8B heads): batch 1 over 2304 keys is fastest at
     // 24-32 splits, batch 4 over ~2k keys at 8, batch 16 over 4k-8k keys at 12;
