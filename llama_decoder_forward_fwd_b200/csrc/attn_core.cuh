@@ -11,9 +11,9 @@
 // heads at each query token, flattened as t*G + h; a chunk holds up to 16 of
 // them (whole tokens when G <= 16, part of one token's heads when G > 16), so
 // each key and value row is read once for all the rows of a chunk. Each of the
-// NW warps takes 32-key groups of the split. Lane j loads the whole key row j into registers and the value slice (dims 4l..4l+3)
-// of all 32 keys, every load issued before the first use, so a group costs one
-// memory round trip. Lane j scores key j for every row against the query rows,
+// NW warps takes 32-key groups of the split. Lane j loads the whole key row j
+// into registers and the value slice (dims 4l..4l+3) of all 32 keys, every load
+// issued before the first use, so a group costs one memory round trip. Lane j scores key j for every row against the query rows,
 // which all lanes read from shared memory as broadcasts; the warp keeps an
 // online softmax (running max and sum, log2 domain) and accumulates P V. The
 // warps' states, then the splits' states (m, l, o), are merged by the
