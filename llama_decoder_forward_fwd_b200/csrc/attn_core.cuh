@@ -13,12 +13,13 @@
 // each key and value row is read once for all the rows of a chunk. Each of the
 // NW warps takes 32-key groups of the split. Lane j loads the whole key row j
 // into registers and the value slice (dims 4l..4l+3) of all 32 keys, every load
-// issued before the first use, so a group costs one memory round trip. Lane j scores key j for every row against the query rows,
-// which all lanes read from shared memory as broadcasts; the warp keeps an
-// online softmax (running max and sum, log2 domain) and accumulates P V. The
-// warps' states, then the splits' states (m, l, o), are merged by the
-// log-sum-exp rule; the split merge is done by whichever CTA of the group
-// finishes last (an atomic counter, no waiting), which also resets the counter.
+// issued before the first use, so a group costs one memory round trip. Lane j
+// scores key j for every row against the query rows, which all lanes read from
+// shared memory as broadcasts; the warp keeps an online softmax (running max
+// and sum, log2 domain) and accumulates P V. The warps' states, then the
+// splits' states (m, l, o), are merged by the log-sum-exp rule; the split merge
+// is done by whichever CTA of the group finishes last (an atomic counter, no
+// waiting), which also resets the counter.
 //
 // Queries, keys and values are read with ld.global.cg: in the fused kernel they
 // were written earlier in the same launch by other CTAs.
