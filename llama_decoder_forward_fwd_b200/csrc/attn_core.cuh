@@ -1,5 +1,6 @@
-// One work item of split-KV decode attention, shared by the single-launch
-// kernel (attn_decode.cu) and the fused decode-step kernel (decode_step.cu).
+// One work item of split-KV decode attention, run by the single-launch kernel
+// of attn_decode.cu (the workspace and the allocation-free entry points; the
+// fused decode step streams its attention through its own ring instead).
 //
 // Causal grouped-query attention of a few new tokens against the KV cache
 // ("Implementación de la atención"; "GQA", "Scaled Dot-Product Attention" and
@@ -21,8 +22,8 @@
 // is done by whichever CTA of the group finishes last (an atomic counter, no
 // waiting), which also resets the counter.
 //
-// Queries, keys and values are read with ld.global.cg: in the fused kernel they
-// were written earlier in the same launch by other CTAs.
+// Queries, keys and values are read with ld.global.cg (L2 only): each byte is
+// used by one CTA, so nothing is gained by keeping it in L1.
 #pragma once
 #include "common.cuh"
 #include "kernels.cuh"
