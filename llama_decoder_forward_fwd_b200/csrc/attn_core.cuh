@@ -22,8 +22,8 @@
 // is done by whichever CTA of the group finishes last (an atomic counter, no
 // waiting), which also resets the counter.
 //
-// Queries, keys and values are read with ld.global.cg (L2 only): each byte is
-// used by one CTA, so nothing is gained by keeping it in L1.
+// Queries, keys and values are read with ld.global.cg (cached in L2 only);
+// each byte is used by one CTA.
 #pragma once
 #include "common.cuh"
 #include "kernels.cuh"
