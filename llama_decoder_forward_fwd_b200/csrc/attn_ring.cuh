@@ -1,13 +1,12 @@
-// Decode attention streamed in 32-key units, shared by the single-launch ring
-// attention kernel (attn_decode_ring.cu) and the fused decode step
-// (decode_step.cu).
+// Decode attention streamed in 32-key units through the fused decode step's
+// shared-memory ring (decode_step.cu).
 //
 // A unit is the K and V tiles of 32 consecutive keys of one (sequence, KV head)
 // group: two 64-dim halves of 32 rows x 128 bytes each for K and for V, loaded by
 // TMA with the 128-byte swizzle into one 16 KB ring stage. A group's keys are
 // 0 .. len (the new token sits at position len), so it has ceil((len + 1) / 32)
 // units, and the units of all groups, in group order, are split evenly over the
-// CTAs. Both kernels compute S = Q K^T and P V with mma.sync m16n8k16 from the
+// CTAs. The step computes S = Q K^T and P V with mma.sync m16n8k16 from the
 // swizzled tiles (the group's query heads padded to 16 rows) and an online
 // softmax in the log2 domain ("Implementación de la atención"; "GQA" and
 // "Scaled Dot-Product Attention" on the llama3.np page).

@@ -2,8 +2,9 @@
 // layer's QKV projection with RoPE and KV-cache append, attention, wo projection
 // with residual, w1/w3 projection with SwiGLU, w2 projection with residual, and
 // the lm_head with greedy argmax) in a single persistent launch with one CTA per
-// SM ("Resumen ..." and "Predicción de tokens" on "Implementación de LLaMA3 en
-// Python puro"; "Transformer Block" on the llama3.np page).
+// SM ("Resumen de una implementación desde cero del modelo LLaMA-3": attention
+// and feed-forward repeated over every layer, then "Predicción de tokens";
+// "手撕Llama3第1层", section 6: the stacked transformer blocks).
 //
 // Why one launch: a decode step streams every weight once (16 GB for the 8B
 // shape) but runs ~160 dependent projections, each only tens of microseconds
