@@ -52,8 +52,8 @@ DEVI uint32_t w_of(const uint4& a, const uint4& b, int i) {
 }
 
 // Order-preserving key of (logit, token id) for a 64-bit atomicMax: a larger
-// logit wins, and among equal logits the lower id ("the highest value is the
-// next token"; ties go to the lowest id).
+// logit wins, and among equal logits the lower id ("Predicción de tokens": the
+// token with the largest logit comes next; ties go to the lowest id).
 DEVI unsigned long long am_key(float v, int idx) {
     uint32_t u = __float_as_uint(v);
     u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);

@@ -147,8 +147,9 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, q_pos: np.ndarray,
     Returns [Tq, H*d] with heads concatenated in head order.
 
     Scores are q.k / sqrt(d) ("Scaled Dot-Product Attention"); a key at a
-    position after the query's is masked to -inf before the softmax ("mask of
-    future tokens"); the output is the softmax-weighted sum of values, then the
+    position after the query's is masked to -inf before the softmax
+    ("Implementación de la atención": scores of future tokens are masked); the
+    output is the softmax-weighted sum of values, then the
     heads are concatenated ("Atención multi-head"). Query head h uses KV head
     floor(h / (H / Hk)) (GQA, "GQA(Grouped-Query Attention)").
     """
