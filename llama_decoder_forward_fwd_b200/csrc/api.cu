@@ -764,7 +764,6 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
                      cudaMemsetAsync(m->gws.done_cnt, 0, 16, m->stream) != cudaSuccess ||
                      cudaMemsetAsync(m->gws.warp_cnt, 0, (size_t)m->gws.tiles_cap * 8 * 4, m->stream) != cudaSuccess)))
         return bail(fail(LLM_ERR_CUDA, "cudaMemsetAsync failed"));
-    if (attn_decode_prepare() != cudaSuccess) return bail(fail(LLM_ERR_CUDA, "attention kernel attributes"));
     if (launch_rope_tables(m->rope_cos, m->rope_sin, c.max_seq_len, d / 2, (double)c.rope_theta, d, m->stream) !=
         cudaSuccess)
         return bail(fail(LLM_ERR_CUDA, "rope table kernel failed"));

@@ -70,7 +70,4 @@ cudaError_t launch_attn_decode(const AttnDecodeArgs& a, bool bf16, cudaStream_t 
     return launch_one<float, 16>(a, s, pdl);
 }
 
-// Nothing to configure: the kernel uses static shared memory only.
-cudaError_t attn_decode_prepare() { return cudaSuccess; }
-
 }  // namespace lfw

@@ -170,7 +170,6 @@ struct AttnDecodePlan {
 };
 AttnDecodePlan attn_decode_plan(int B, int T, int H, int Hk, int d, int max_keys, int num_sms);
 cudaError_t launch_attn_decode(const AttnDecodeArgs& a, bool bf16, cudaStream_t s, bool pdl);
-cudaError_t attn_decode_prepare();
 
 // ---- fused decode step (bf16): the whole model in one persistent launch ----
 struct DecodeStepArgs {
