@@ -102,3 +102,19 @@ def test_split_kv_workspace_follows_the_16_row_work_items(lib, B, T, H, Hk, d, i
     part = items * rows * 64 * (d + 4) * 4
     expect = ((part + 255) & ~255) + items * 4
     assert lib.llm_op_attention_decode_workspace(B, T, H, Hk, d) == expect
+
+
+@pytest.mark.parametrize("n_kv_heads", [32, 8, 2, 1])
+def test_any_query_group_size_passes_config_validation(lib, n_kv_heads):
+    """Multi-head, grouped-query and multi-query configs are all valid: with no
+    weights given, init gets past the config checks and stops at the missing
+    weights (before touching a device); a head count that does not divide is not."""
+    import seeded_inputs as S
+    shape = S.WORKLOADS["llama3-8b-bf16-b1-p2048-g256"].shape
+    w = L.llm_weights()
+    h = ctypes.c_void_p()
+    cfg = L.make_config(shape.replace(n_kv_heads=n_kv_heads), max_batch=1)
+    assert lib.llm_model_init(ctypes.byref(cfg), ctypes.byref(w), None, ctypes.byref(h)) == L.LLM_ERR_NULL_PTR
+    assert b"weight" in lib.llm_last_error()
+    cfg = L.make_config(shape.replace(n_kv_heads=3), max_batch=1)
+    assert lib.llm_model_init(ctypes.byref(cfg), ctypes.byref(w), None, ctypes.byref(h)) == L.LLM_ERR_BAD_CONFIG
