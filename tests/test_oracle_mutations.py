@@ -6,6 +6,7 @@ against that copy in a separate process, and requires them to fail. An
 unmodified copy must pass, so a broken copy mechanism cannot make every mutant
 look caught. The mistakes are planted in the oracle only, on the CPU.
 """
+import concurrent.futures as cf
 import os
 import shutil
 import subprocess
@@ -37,8 +38,7 @@ MUTATIONS = {
 }
 
 
-def _run_pins(tmp_path, mutation):
-    tree = tmp_path / "tree"
+def _run_pins(tree, mutation):
     for d in ("oracle", "seeded_inputs"):
         shutil.copytree(os.path.join(ROOT, d), tree / d, ignore=shutil.ignore_patterns("__pycache__"))
     (tree / "tests").mkdir()
@@ -52,17 +52,29 @@ def _run_pins(tmp_path, mutation):
         assert src.count(old) == 1, f"mutation site not unique or missing: {old!r}"
         src_path.write_text(src.replace(old, new))
     env = {k: v for k, v in os.environ.items() if k != "PYTHONPATH"}
+    env["OMP_NUM_THREADS"] = "1"   # the copies run side by side
     r = subprocess.run([sys.executable, "-m", "pytest", "tests/test_oracle_pins.py", "-q", "-x", "-p", "no:cacheprovider"],
                        cwd=tree, env=env, capture_output=True, text=True, timeout=600)
     return r.returncode, r.stdout[-2000:]
 
 
-def test_unmodified_copy_passes(tmp_path):
-    rc, out = _run_pins(tmp_path, None)
+@pytest.fixture(scope="module")
+def results(tmp_path_factory):
+    """Exit code and output tail of the pins on the unmodified copy (key None) and
+    on every mutant, run as independent processes side by side."""
+    cases = [None] + sorted(MUTATIONS)
+    with cf.ThreadPoolExecutor(max_workers=max(1, min(8, os.cpu_count() or 1))) as ex:
+        futs = {name: ex.submit(_run_pins, tmp_path_factory.mktemp("tree"),
+                                None if name is None else MUTATIONS[name]) for name in cases}
+        return {name: f.result() for name, f in futs.items()}
+
+
+def test_unmodified_copy_passes(results):
+    rc, out = results[None]
     assert rc == 0, out
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
-def test_planted_mistake_fails_a_pin(tmp_path, name):
-    rc, out = _run_pins(tmp_path, MUTATIONS[name])
+def test_planted_mistake_fails_a_pin(results, name):
+    rc, out = results[name]
     assert rc == 1, f"{name}: pins still pass (exit {rc})\n{out}"
