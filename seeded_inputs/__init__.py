@@ -105,6 +105,12 @@ WORKLOADS: Dict[str, Workload] = {
         shape=_LLAMA3_8B.replace(max_seq_len=8192),
         batch=1, prompt_len=0, decode_steps=128, input_kind="kv_prefilled",
         kv_len_range=(8064, 8064)),
+    # Multi-query variant of the Llama-3-8B shape (one KV head for all 32 query
+    # heads), otherwise the benchmark's configuration.
+    "llama3-8b-mqa-bf16-b1-p2048-g256": Workload(
+        name="llama3-8b-mqa-bf16-b1-p2048-g256",
+        shape=_LLAMA3_8B.replace(n_kv_heads=1, max_seq_len=2048 + 256),
+        batch=1, prompt_len=2048, decode_steps=256, input_kind="tokens"),
     # Llama-2-7B-shaped multi-head (no GQA) model, batch 8.
     "llama2-7b-mha-bf16-b8-p1024-g256": Workload(
         name="llama2-7b-mha-bf16-b8-p1024-g256",
