@@ -109,6 +109,7 @@ def test_special_tokens_only_where_allowed():
 
 def test_round_trip_on_random_text():
     tok = T.Tokenizer(_trained_vocab(CORPUS, 120))
+    assert tok.decode(tok.encode(GOLD["round_trip_text"])) == GOLD["round_trip_text"]   # the page's own check
     rng = random.Random(0)
     alphabet = "abcdefghij ,.!?'\n\t0123456789ÄéßñЖ中文😀 " + "the answer "
     for _ in range(200):
