@@ -36,12 +36,16 @@ Sources (page title, then section), all restated in this module's own words:
 * "LLaMA2" (downcodes): RoPE as a rotation whose q.k product depends only on the
   position offset; GQA/MQA share K/V heads among query heads; the KV cache.
 
-``OracleModel(..., bf16_activations=True)`` is the same computation with the
-activations rounded to bf16 (nearest, ties to even) at the points where a bf16
-implementation stores them: each projection input h * norm weight (the norm's
-1/rms scale applied after the product), q, k and v after RoPE, the attention
-output and the SwiGLU output. It exists to state what that storage policy alone
-does to the result at depth; every other value stays exact.
+``OracleModel(..., rounding=points)`` is the same computation with the
+activations rounded to bf16 (nearest, ties to even) at the named points where a
+bf16 implementation can store them (``BF16_POINTS``): "x", each projection input
+h * norm weight (the norm's 1/rms scale applied after the product); "q", "k" and
+"v" after RoPE (k and v are the KV cache); "o", the attention output; "g", the
+SwiGLU output. ``bf16_activations=True`` rounds at all of them. ``BF16_FORCED``
+names the points no bf16 tensor-core implementation with a bf16 KV cache can
+avoid: the inputs of the four projections (x, o, g: the bf16 operands of the
+matrix products) and the cache (k, v). These modes exist to state what a storage
+policy alone does to the result at depth; every other value stays exact.
 
 Readings where the pages are silent or garbled (each is also listed in the
 design notes): RoPE rotates interleaved adjacent pairs (2i, 2i+1) with angle
@@ -59,9 +63,13 @@ import numpy as np
 import torch
 
 __all__ = [
-    "f64", "round_bf16", "rmsnorm", "rope_tables", "rope", "softmax", "silu", "attention",
-    "swiglu_ffn", "argmax_first", "OracleModel",
+    "BF16_POINTS", "BF16_FORCED", "f64", "round_bf16", "rmsnorm", "rope_tables", "rope", "softmax", "silu",
+    "attention", "swiglu_ffn", "argmax_first", "OracleModel",
 ]
+
+
+BF16_POINTS = frozenset({"x", "q", "k", "v", "o", "g"})
+BF16_FORCED = frozenset({"x", "k", "v", "o", "g"})
 
 
 def f64(t) -> np.ndarray:
@@ -195,9 +203,12 @@ class OracleModel:
     """
 
     def __init__(self, shape, glob: Dict, layers, batch: int, keep_f64_layers: bool = True,
-                 bf16_activations: bool = False):
+                 bf16_activations: bool = False, rounding=None):
         self.s = shape
-        self.bf16 = bf16_activations
+        if rounding is None:
+            rounding = BF16_POINTS if bf16_activations else frozenset()
+        assert set(rounding) <= BF16_POINTS, f"unknown rounding points {set(rounding) - BF16_POINTS}"
+        self.rounding = frozenset(rounding)
         self.glob = glob
         self._layers = layers
         self._cache64: Dict[int, Dict[str, np.ndarray]] = {}
@@ -256,25 +267,25 @@ class OracleModel:
             pos = pos0[b] + np.arange(T)
             q = (x[b] @ w["wq"].T).reshape(T, H, d)
             k = (x[b] @ w["wk"].T).reshape(T, Hk, d)
-            v = r((x[b] @ w["wv"].T).reshape(T, Hk, d))
-            q = r(rope(q, pos, s.rope_theta))
-            k = r(rope(k, pos, s.rope_theta))
+            v = r((x[b] @ w["wv"].T).reshape(T, Hk, d), "v")
+            q = r(rope(q, pos, s.rope_theta), "q")
+            k = r(rope(k, pos, s.rope_theta), "k")
             assert self.K[l][b].shape[0] == pos0[b], "cache length and position disagree"
             self.K[l][b] = np.concatenate([self.K[l][b], k], axis=0)
             self.V[l][b] = np.concatenate([self.V[l][b], v], axis=0)
             kpos = np.arange(self.K[l][b].shape[0])
-            out[b] = r(attention(q, self.K[l][b], self.V[l][b], pos, kpos))
+            out[b] = r(attention(q, self.K[l][b], self.V[l][b], pos, kpos), "o")
         h = h + out @ w["wo"].T
         x = self._norm_in(h, w["ffn_norm"])
-        return h + r(silu(x @ w["w1"].T) * (x @ w["w3"].T)) @ w["w2"].T
+        return h + r(silu(x @ w["w1"].T) * (x @ w["w3"].T), "g") @ w["w2"].T
 
-    def _round(self, a: np.ndarray) -> np.ndarray:
-        return round_bf16(a) if self.bf16 else a
+    def _round(self, a: np.ndarray, point: str) -> np.ndarray:
+        return round_bf16(a) if point in self.rounding else a
 
     def _norm_in(self, h: np.ndarray, wn: np.ndarray) -> np.ndarray:
-        """RMSNorm(h) * wn; with bf16 activations, h * wn is stored in bf16 and the
+        """RMSNorm(h) * wn; when "x" is rounded, h * wn is stored in bf16 and the
         1/rms scale is applied to it afterwards (the same value in exact arithmetic)."""
-        if not self.bf16:
+        if "x" not in self.rounding:
             return rmsnorm(h, wn, self.s.norm_eps)
         rinv = 1.0 / np.sqrt(np.mean(h * h, axis=-1, keepdims=True) + self.s.norm_eps)
         return round_bf16(h * wn) * rinv

@@ -13,6 +13,7 @@ import math
 import os
 
 import numpy as np
+import pytest
 import torch
 
 import oracle as O
@@ -371,3 +372,32 @@ def test_bf16_emulation_rounds_where_stated_and_stays_close():
         assert 1e-5 < d < 1e-2, d
     d = np.linalg.norm(le - lp) / np.linalg.norm(lp)
     assert 1e-5 < d < 1e-2, d
+
+
+def test_bf16_rounding_points_round_only_where_named():
+    """Each named storage point rounds its own value and nothing else: the cache
+    holds bf16 values exactly when k (or v) is named, and every point alone moves
+    the result by a small, nonzero amount; the forced set is every point but q."""
+    assert O.BF16_FORCED == O.BF16_POINTS - {"q"}
+    shape = S.ModelShape(dim=64, n_layers=2, n_heads=4, n_kv_heads=2, head_dim=16, ffn_hidden=96,
+                         vocab=50, max_seq_len=32, norm_eps=1e-5, rope_theta=10000.0, dtype="bf16",
+                         tie_embeddings=False)
+    glob, layers = S.make_weights(shape, 13)
+    tok = S.make_tokens(13, 1, 7, shape.vocab).numpy()
+    plain = O.OracleModel(shape, glob, layers, 1)
+    _, lp = plain.prefill(tok)
+    logits = {}
+    for p in sorted(O.BF16_POINTS):
+        m = O.OracleModel(shape, glob, layers, 1, rounding={p})
+        _, logits[p] = m.prefill(tok)
+        for l in range(shape.n_layers):
+            for cache, name in ((m.K[l][0], "k"), (m.V[l][0], "v")):
+                assert np.array_equal(O.round_bf16(cache), cache) == (p == name), (p, name)
+        d = np.linalg.norm(logits[p] - lp) / np.linalg.norm(lp)
+        assert 1e-6 < d < 1e-2, (p, d)
+    for a in logits:
+        for b in logits:
+            if a < b:
+                assert not np.array_equal(logits[a], logits[b]), (a, b)
+    with pytest.raises(AssertionError):
+        O.OracleModel(shape, glob, layers, 1, rounding={"w"})
