@@ -277,22 +277,46 @@ int llm_op_attention_decode(const void* q, const void* kcache, const void* vcach
                             size_t workspace_bytes, void* stream);
 
 /*
+ * Decode attention of one new token per sequence on the tensor cores, as the
+ * bf16 decode path runs it ("Implementación de la atención"; llama3.np "GQA",
+ * "Scaled Dot-Product Attention", "KV cache"): out[b][h] = softmax over keys
+ * 0..pos0[b] of q[b][h] . K[b][h/G][j] / sqrt(128), times V[b][h/G][j].
+ *   q, out: [B][H*128] bf16; kcache, vcache: [B][Hk][S_max][128] bf16 holding
+ *   positions 0..pos0[b] (the new token's key and value included); pos0: [B]
+ *   int32 (0 <= pos0[b] < S_max). G = H / Hk must be at most 8. Device
+ *   pointers, 16-byte aligned, owned by the caller; no workspace: a thread-block
+ *   cluster per (sequence, KV head) streams 32-key K/V tiles by TMA and merges
+ *   its CTAs' partial results in distributed shared memory. The probabilities
+ *   enter the P V product rounded to bf16 (fp32 accumulation).
+ *   Errors: LLM_ERR_NULL_PTR, LLM_ERR_BAD_ARG (shape, alignment),
+ *   LLM_ERR_UNSUPPORTED (G > 8), LLM_ERR_CUDA.
+ */
+int llm_op_attention_decode_cluster(const void* q, const void* kcache, const void* vcache,
+                                    const int32_t* pos0, void* out, int B, int H, int Hk,
+                                    int S_max, void* stream);
+
+/*
  * The split-KV decode attention of llm_op_attention_decode, for callers that
  * cannot allocate device memory: code running while a stream is captured into
  * a CUDA graph (cudaMalloc cannot be captured), plug-ins whose host
  * application owns every device allocation, and latency-critical loops where
  * an allocation could synchronise the device. The pages have no counterpart:
  * this is a deployment convenience, not a step of the decoder.
- *   Same arguments and results as llm_op_attention_decode, without the
- *   workspace: the scratch is a fixed array inside the library (8 MiB of
- *   per-split partial results and 4096 merge counters), held by every GPU that
- *   loads the library until the process exits. The call allocates nothing
- *   (no cudaMalloc, cudaFree or allocating library routine).
+ *   Same arguments, checks, split plan (from S_max) and results as
+ *   llm_op_attention_decode, without the workspace: the scratch is a fixed
+ *   array inside the library (8 MiB of per-split partial results and 4096 merge
+ *   counters), held by every GPU that loads the library until the process
+ *   exits. The call allocates nothing (no cudaMalloc, cudaFree or allocating
+ *   library routine).
  *   Shapes that need more scratch than that return LLM_ERR_BAD_ARG before
- *   anything is queued (at B = 1..7 with 32 query heads, 8 KV heads and
- *   head_dim 128 they fit).
- *   The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   anything is queued: a call needs B * Hk * ceil(T * G / rows) * rows *
+ *   splits * (d + 4) floats (G = H / Hk; rows = 16 when G >= 16, else
+ *   G * min(floor(16 / G), T); splits as llm_op_attention_decode plans them). With 32 query heads,
+ *   8 KV heads and head_dim 128, one new token per sequence fits for every
+ *   B <= 16 and S_max <= 16384.
+ *   The first call in a CUDA context (once per device, and again after
+ *   cudaDeviceReset) looks up the array's device address (cudaGetSymbolAddress);
+ *   make that first call before any stream capture.
  *   Every call uses the same array and zeroes its counters first, so calls
  *   whose kernels may overlap on the GPU (other streams, other host threads)
  *   race with each other and must not be issued.

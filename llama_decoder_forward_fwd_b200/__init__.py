@@ -80,6 +80,7 @@ _SIGS = {
     "llm_op_attention_decode_workspace": (_sz, [_i, _i, _i, _i, _i]),
     "llm_op_attention_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]),
     "llm_op_attention_decode_static": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "llm_op_attention_decode_cluster": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
 }
 
 
@@ -303,6 +304,14 @@ class Model:
             self.free()
         except Exception:
             pass
+
+
+def llm_op_attention_decode_cluster(q, kc, vc, pos0, out, stream=None):
+    """Single-token decode attention on the tensor cores (bf16, head_dim 128, no workspace)."""
+    B, T, H, d = q.shape
+    Hk, S = kc.shape[1], kc.shape[2]
+    check(load().llm_op_attention_decode_cluster(_ptr(q), _ptr(kc), _ptr(vc), _ptr(pos0), _ptr(out), B, H, Hk, S,
+                                                 _stream_ptr(stream)))
 
 
 def llm_op_attention_decode_static(q, kc, vc, pos0, out, stream=None):

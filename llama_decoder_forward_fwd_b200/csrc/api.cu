@@ -102,6 +102,7 @@ __device__ uint32_t g_op_err;  // device error word of the single-operation entr
 }  // namespace
 
 int lfw::set_error(int code, const char* msg) { return fail(code, "%s", msg); }
+int lfw::current_num_sms() { return num_sms_current(); }
 
 struct llm_model {
     llm_config cfg;
@@ -137,6 +138,8 @@ struct llm_model {
     std::vector<int> host_len;
     // tensor maps (bf16 models)
     CUtensorMap tm_hw, tm_o, tm_g, tm_kc, tm_vc, tm_head;
+    CUtensorMap tm_k32, tm_v32;  // the K and V caches in 32-row boxes (decode attention units)
+    bool kv32_ok = false;
     std::vector<CUtensorMap> tm_w;
     bool gemm_ok = false;
     // fused decode step (bf16): device copies of the weight tensor maps and norm
@@ -316,21 +319,24 @@ Epi base_epi(llm_model* m, int M, int T) {
     return e;
 }
 
-// Decoder layers over M = B*T token rows; h/hw/ss hold the embedding output.
-int run_layers(llm_model* m, int B, int T, int max_keys) {
+// The launches of one layer, in order.
+enum { PH_QKV, PH_ATTN, PH_WO, PH_W13, PH_W2, PH_PER_LAYER };
+
+// Phase p (PH_QKV .. PH_W2) of layer l over M = B*T token rows, each as its
+// own launch. *nparts: partial sums of h^2 that describe the current RMSNorm input
+// hw (set by the residual phases).
+int run_phase(llm_model* m, int l, int p, int B, int T, int max_keys, int* nparts) {
     const llm_config& c = m->cfg;
     const int M = B * T, D = c.dim, H = c.n_heads, Hk = c.n_kv_heads, d = c.head_dim, F = c.ffn_hidden;
-    int nparts = 1;
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
-    for (int l = 0; l < c.n_layers; ++l) {
-        const LayerW& w = m->L[l];
-        char* kbase = reinterpret_cast<char*>(m->kc) + (size_t)l * m->layer_elems * m->esz;
-        char* vbase = reinterpret_cast<char*>(m->vc) + (size_t)l * m->layer_elems * m->esz;
-        // QKV + RoPE + cache append
-        {
+    const LayerW& w = m->L[l];
+    char* kbase = reinterpret_cast<char*>(m->kc) + (size_t)l * m->layer_elems * m->esz;
+    char* vbase = reinterpret_cast<char*>(m->vc) + (size_t)l * m->layer_elems * m->esz;
+    switch (p) {
+        case PH_QKV: {  // QKV + RoPE + cache append
             Epi e = base_epi(m, M, T);
             e.kind = EPI_QKV_ROPE;
-            e.norm = norm_in(m, nparts);
+            e.norm = norm_in(m, *nparts);
             e.pos0 = m->seq_len;
             e.rope_cos = m->rope_cos;
             e.rope_sin = m->rope_sin;
@@ -344,56 +350,70 @@ int run_layers(llm_model* m, int B, int T, int max_keys) {
             const void* W[3] = {w.wq, w.wk, w.wv};
             const int seg[3] = {H * d, Hk * d, Hk * d};
             const int tms[3] = {TM_WQ, TM_WK, TM_WV};
-            int rc = project(m, l, EPI_QKV_ROPE, LLM_K_QKV, m->hw, &m->tm_hw, D, (H + 2 * Hk) * d, W, seg, tms, e, M, nullptr);
-            if (rc) return rc;
+            return project(m, l, EPI_QKV_ROPE, LLM_K_QKV, m->hw, &m->tm_hw, D, (H + 2 * Hk) * d, W, seg, tms, e, M,
+                           nullptr);
         }
-        // attention
-        {
-        KTimer attn_timer(m, LLM_K_ATTN);
-        if (T > 1 && m->bf16 && d == 128) {
-            AttnPrefillArgs a;
-            a.tmK = &m->tm_kc;
-            a.tmV = &m->tm_vc;
-            a.row_base = (long long)l * c.max_batch * Hk * c.max_seq_len;
-            a.S_max = c.max_seq_len;
-            a.q = reinterpret_cast<const __nv_bfloat16*>(m->q);
-            a.out = reinterpret_cast<__nv_bfloat16*>(m->o);
-            a.pos0 = m->seq_len;
-            a.B = B;
-            a.T = T;
-            a.H = H;
-            a.Hk = Hk;
-            a.scale_log2 = scale_log2;
-            a.err = m->d_err;
-            CK(launch_attn_prefill(a, m->stream, m->pdl));
-        } else {
-            const AttnDecodePlan p = attn_decode_plan(B, T, H, Hk, d, max_keys, m->num_sms);
-            if (p.part_floats > m->attn_ws_floats || p.counters > m->attn_cnt_n)
-                return fail(LLM_ERR_UNSUPPORTED, "attention scratch too small for this call");
-            AttnDecodeArgs a;
-            a.q = m->q;
-            a.kc = kbase;
-            a.vc = vbase;
-            a.out = m->o;
-            a.pos0 = m->seq_len;
-            a.B = B;
-            a.T = T;
-            a.H = H;
-            a.Hk = Hk;
-            a.d = d;
-            a.S_max = c.max_seq_len;
-            a.n_splits = p.n_splits;
-            a.rows = p.rows;
-            a.n_qchunks = p.n_qchunks;
-            a.ws_part = m->attn_ws;
-            a.ws_count = m->attn_cnt;
-            a.scale_log2 = scale_log2;
-            a.err = m->d_err;
-            CK(launch_attn_decode(a, m->bf16, m->stream, m->pdl));
+        case PH_ATTN: {
+            KTimer attn_timer(m, LLM_K_ATTN);
+            if (T > 1 && m->bf16 && d == 128) {
+                AttnPrefillArgs a;
+                a.tmK = &m->tm_kc;
+                a.tmV = &m->tm_vc;
+                a.row_base = (long long)l * c.max_batch * Hk * c.max_seq_len;
+                a.S_max = c.max_seq_len;
+                a.q = reinterpret_cast<const __nv_bfloat16*>(m->q);
+                a.out = reinterpret_cast<__nv_bfloat16*>(m->o);
+                a.pos0 = m->seq_len;
+                a.B = B;
+                a.T = T;
+                a.H = H;
+                a.Hk = Hk;
+                a.scale_log2 = scale_log2;
+                a.err = m->d_err;
+                CK(launch_attn_prefill(a, m->stream, m->pdl));
+            } else if (T == 1 && m->bf16 && m->kv32_ok && attn_cluster_size(B, H, Hk, d, m->num_sms) > 0) {
+                AttnClusterArgs a;
+                a.q = reinterpret_cast<const __nv_bfloat16*>(m->q);
+                a.out = reinterpret_cast<__nv_bfloat16*>(m->o);
+                a.pos0 = m->seq_len;
+                a.B = B;
+                a.H = H;
+                a.Hk = Hk;
+                a.S_max = c.max_seq_len;
+                a.row_base = (long long)l * c.max_batch * Hk * c.max_seq_len;
+                a.rows_per_seq = (long long)Hk * c.max_seq_len;
+                a.cs = attn_cluster_size(B, H, Hk, d, m->num_sms);
+                a.scale_log2 = scale_log2;
+                a.err = m->d_err;
+                CK(launch_attn_cluster(a, &m->tm_k32, &m->tm_v32, m->stream));
+            } else {
+                const AttnDecodePlan pl = attn_decode_plan(B, T, H, Hk, d, max_keys, m->num_sms);
+                if (pl.part_floats > m->attn_ws_floats || pl.counters > m->attn_cnt_n)
+                    return fail(LLM_ERR_UNSUPPORTED, "attention scratch too small for this call");
+                AttnDecodeArgs a;
+                a.q = m->q;
+                a.kc = kbase;
+                a.vc = vbase;
+                a.out = m->o;
+                a.pos0 = m->seq_len;
+                a.B = B;
+                a.T = T;
+                a.H = H;
+                a.Hk = Hk;
+                a.d = d;
+                a.S_max = c.max_seq_len;
+                a.n_splits = pl.n_splits;
+                a.rows = pl.rows;
+                a.n_qchunks = pl.n_qchunks;
+                a.ws_part = m->attn_ws;
+                a.ws_count = m->attn_cnt;
+                a.scale_log2 = scale_log2;
+                a.err = m->d_err;
+                CK(launch_attn_decode(a, m->bf16, m->stream, m->pdl));
+            }
+            return LLM_OK;
         }
-        }
-        // wo + residual; writes the ffn_norm input
-        {
+        case PH_WO: {  // wo + residual; writes the ffn_norm input
             Epi e = base_epi(m, M, T);
             e.kind = EPI_RESID;
             e.h = m->h;
@@ -405,24 +425,20 @@ int run_layers(llm_model* m, int B, int T, int max_keys) {
             const void* W[3] = {w.wo, nullptr, nullptr};
             const int seg[3] = {D, 0, 0};
             const int tms[3] = {TM_WO, -1, -1};
-            int rc = project(m, l, EPI_RESID, LLM_K_WO, m->o, &m->tm_o, H * d, D, W, seg, tms, e, M, &nparts);
-            if (rc) return rc;
+            return project(m, l, EPI_RESID, LLM_K_WO, m->o, &m->tm_o, H * d, D, W, seg, tms, e, M, nparts);
         }
-        // w1, w3 + SwiGLU
-        {
+        case PH_W13: {  // w1, w3 + SwiGLU
             Epi e = base_epi(m, M, T);
             e.kind = EPI_SWIGLU;
-            e.norm = norm_in(m, nparts);
+            e.norm = norm_in(m, *nparts);
             e.g_out = m->g;
             e.F = F;
             const void* W[3] = {w.w1, w.w3, nullptr};
             const int seg[3] = {F, 0, 0};
             const int tms[3] = {TM_W1, TM_W3, -1};
-            int rc = project(m, l, EPI_SWIGLU, LLM_K_W13, m->hw, &m->tm_hw, D, F, W, seg, tms, e, M, nullptr);
-            if (rc) return rc;
+            return project(m, l, EPI_SWIGLU, LLM_K_W13, m->hw, &m->tm_hw, D, F, W, seg, tms, e, M, nullptr);
         }
-        // w2 + residual; writes the next norm's input
-        {
+        default: {  // w2 + residual; writes the next norm's input
             Epi e = base_epi(m, M, T);
             e.kind = EPI_RESID;
             e.h = m->h;
@@ -434,7 +450,19 @@ int run_layers(llm_model* m, int B, int T, int max_keys) {
             const void* W[3] = {w.w2, nullptr, nullptr};
             const int seg[3] = {D, 0, 0};
             const int tms[3] = {TM_W2, -1, -1};
-            int rc = project(m, l, EPI_RESID, LLM_K_W2, m->g, &m->tm_g, F, D, W, seg, tms, e, M, &nparts);
+            return project(m, l, EPI_RESID, LLM_K_W2, m->g, &m->tm_g, F, D, W, seg, tms, e, M, nparts);
+        }
+    }
+}
+
+// Decoder layers over M = B*T token rows; h/hw/ss hold the embedding output.
+int run_layers(llm_model* m, int B, int T, int max_keys) {
+    const llm_config& c = m->cfg;
+    const int M = B * T, D = c.dim;
+    int nparts = 1;
+    for (int l = 0; l < c.n_layers; ++l) {
+        for (int p = 0; p < PH_PER_LAYER; ++p) {
+            const int rc = run_phase(m, l, p, B, T, max_keys, &nparts);
             if (rc) return rc;
         }
         if (m->taps)
@@ -534,16 +562,9 @@ DecodeStepPlan fused_plan(const llm_model* m, int B, int max_keys) {
                             c.has_embed_and_head, max_keys, m->num_sms, m->smem_optin);
 }
 
-// One decode step of every sequence b < B as a single fused launch (token ids,
-// or hidden states for a bare layer stack).
-int run_fused_step(llm_model* m, int B, const int32_t* tok, const float* h_in, float* h_out, int32_t* next,
-                   float* logits) {
+// Arguments of the fused decode step for B sequences.
+DecodeStepArgs ds_args(llm_model* m, int B, const DecodeStepPlan& p) {
     const llm_config& c = m->cfg;
-    const DecodeStepPlan p = fused_plan(m, B, max_keys_after(m, B, 1));
-    if (!p.supported) return fail(LLM_ERR_UNSUPPORTED, "fused decode step does not support this shape");
-    if (p.part_floats > m->gws.part_floats || p.tiles > m->gws.tiles_cap || p.attn_part_floats > m->attn_ws_floats ||
-        p.attn_counters > m->attn_cnt_n)
-        return fail(LLM_ERR_UNSUPPORTED, "fused decode step scratch too small for this call");
     DecodeStepArgs a;
     a.B = B;
     a.D = c.dim;
@@ -560,11 +581,6 @@ int run_fused_step(llm_model* m, int B, const int32_t* tok, const float* h_in, f
     a.n_stages = p.n_stages;
     a.xs_bytes = p.xs_bytes;
     for (int i = 0; i < 5; ++i) a.max_pieces[i] = p.max_pieces[i];
-    a.tok = tok;
-    a.h_in = h_in;
-    a.h_out = h_out;
-    a.next = next;
-    a.logits = logits;
     a.tmaps = m->d_tmaps;
     a.norms = m->d_norms;
     a.tok_emb = m->tok_emb;
@@ -587,6 +603,30 @@ int run_fused_step(llm_model* m, int B, const int32_t* tok, const float* h_in, f
     a.attn_cnt = m->attn_cnt;
     a.bar = m->ds_bar;
     a.err = m->d_err;
+    return a;
+}
+
+int ds_check(llm_model* m, const DecodeStepPlan& p) {
+    if (!p.supported) return fail(LLM_ERR_UNSUPPORTED, "fused decode kernel does not support this shape");
+    if (p.part_floats > m->gws.part_floats || p.tiles > m->gws.tiles_cap || p.attn_part_floats > m->attn_ws_floats ||
+        p.attn_counters > m->attn_cnt_n)
+        return fail(LLM_ERR_UNSUPPORTED, "fused decode kernel scratch too small for this call");
+    return LLM_OK;
+}
+
+// One decode step of every sequence b < B as a single fused launch (token ids,
+// or hidden states for a bare layer stack).
+int run_fused_step(llm_model* m, int B, const int32_t* tok, const float* h_in, float* h_out, int32_t* next,
+                   float* logits) {
+    const DecodeStepPlan p = fused_plan(m, B, max_keys_after(m, B, 1));
+    const int rc = ds_check(m, p);
+    if (rc) return rc;
+    DecodeStepArgs a = ds_args(m, B, p);
+    a.tok = tok;
+    a.h_in = h_in;
+    a.h_out = h_out;
+    a.next = next;
+    a.logits = logits;
     KTimer timer(m, LLM_K_STEP);
     CK(cudaMemsetAsync(m->ds_bar, 0, 4, m->stream));
     CK(launch_decode_step(a, p, m->stream));
@@ -760,6 +800,10 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
         cudaMemsetAsync(m->seq_len, 0, (size_t)c.max_batch * 4, m->stream) != cudaSuccess ||
         cudaMemsetAsync(m->d_err, 0, 64, m->stream) != cudaSuccess ||
         cudaMemsetAsync(m->ss, 0, (size_t)parts * Mx * 4, m->stream) != cudaSuccess ||
+        // attention reads whole 32-key tiles: positions past a sequence's length are
+        // masked, and zeroed here so that they never hold a non-finite pattern
+        cudaMemsetAsync(m->kc, 0, (size_t)c.n_layers * m->layer_elems * es, m->stream) != cudaSuccess ||
+        cudaMemsetAsync(m->vc, 0, (size_t)c.n_layers * m->layer_elems * es, m->stream) != cudaSuccess ||
         (m->bf16 && (cudaMemsetAsync(m->gws.am_best, 0, 16 * 8, m->stream) != cudaSuccess ||
                      cudaMemsetAsync(m->gws.done_cnt, 0, 16, m->stream) != cudaSuccess ||
                      cudaMemsetAsync(m->gws.warp_cnt, 0, (size_t)m->gws.tiles_cap * 8 * 4, m->stream) != cudaSuccess)))
@@ -794,8 +838,10 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
                      F % (GEMM_BN / 2) == 0 && D % GEMM_BK == 0 && F % GEMM_BK == 0 && (H * d) % GEMM_BK == 0;
         if (d == 128) {
             const uint64_t rows = (uint64_t)c.n_layers * c.max_batch * Hk * c.max_seq_len;
-            if (!make_tmap(&m->tm_kc, m->kc, d, rows, 64, 64) || !make_tmap(&m->tm_vc, m->vc, d, rows, 64, 64))
+            if (!make_tmap(&m->tm_kc, m->kc, d, rows, 64, 64) || !make_tmap(&m->tm_vc, m->vc, d, rows, 64, 64) ||
+                !make_tmap(&m->tm_k32, m->kc, d, rows, 64, 32) || !make_tmap(&m->tm_v32, m->vc, d, rows, 64, 32))
                 return bail(fail(LLM_ERR_CUDA, "cuTensorMapEncodeTiled (KV cache) failed"));
+            m->kv32_ok = true;
         }
     }
     // Fused decode step: supported shapes only, sized for every batch size at the
@@ -839,15 +885,8 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
             const size_t ntm = (size_t)c.n_layers * TM_PER_LAYER + 3;
             std::vector<CUtensorMap> tms(m->tm_w);
             tms.push_back(c.has_embed_and_head ? m->tm_head : m->tm_w[0]);
-            {
-                // the whole K and V caches as [rows][head_dim], 32-row boxes (attention units)
-                const uint64_t rows = (uint64_t)c.n_layers * c.max_batch * Hk * c.max_seq_len;
-                CUtensorMap k32, v32;
-                if (!make_tmap(&k32, m->kc, d, rows, 64, 32) || !make_tmap(&v32, m->vc, d, rows, 64, 32))
-                    return bail(fail(LLM_ERR_CUDA, "cuTensorMapEncodeTiled (KV cache, fused step) failed"));
-                tms.push_back(k32);
-                tms.push_back(v32);
-            }
+            tms.push_back(m->tm_k32);  // the whole K and V caches, 32-row boxes (attention units)
+            tms.push_back(m->tm_v32);
             std::vector<const void*> norms;
             for (int l = 0; l < c.n_layers; ++l) {
                 norms.push_back(m->L[l].attn_norm);
@@ -1146,20 +1185,9 @@ int llm_op_gemv_bf16(const void* x, const void* W, float* y, int M, int N, int K
     return LLM_OK;
 }
 
-static int attn_common_check(const void* q, const void* kc, const void* vc, const int32_t* pos0, const void* out, int B,
-                             int T, int H, int Hk, int d, int S_max, int dtype) {
-    if (!q || !kc || !vc || !pos0 || !out) return fail(LLM_ERR_NULL_PTR, "NULL operand");
-    if (B < 1 || T < 1 || H < 1 || Hk < 1 || H % Hk != 0 || S_max < 1 || d < 8 || d % 8 != 0 || d > 128)
-        return fail(LLM_ERR_BAD_ARG, "bad attention shape");
-    if (dtype != LLM_F32 && dtype != LLM_BF16) return fail(LLM_ERR_BAD_ARG, "bad dtype");
-    if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(out))
-        return fail(LLM_ERR_BAD_ARG, "operands must be 16-byte aligned");
-    return LLM_OK;
-}
-
 int llm_op_attention_prefill(const void* q, const void* kcache, const void* vcache, const int32_t* pos0, void* out,
                              int B, int T, int H, int Hk, int d, int S_max, int dtype, void* stream) {
-    int rc = attn_common_check(q, kcache, vcache, pos0, out, B, T, H, Hk, d, S_max, dtype);
+    int rc = lfw::attn_op_check(q, kcache, vcache, pos0, out, B, T, H, Hk, d, S_max, dtype);
     if (rc) return rc;
     if (dtype != LLM_BF16 || d != 128) return fail(LLM_ERR_UNSUPPORTED, "flash kernel needs bf16 and d == 128");
     CUtensorMap tk, tv;
@@ -1193,7 +1221,7 @@ size_t llm_op_attention_decode_workspace(int B, int T, int H, int Hk, int d) {
 int llm_op_attention_decode(const void* q, const void* kcache, const void* vcache, const int32_t* pos0, void* out,
                             int B, int T, int H, int Hk, int d, int S_max, int dtype, void* workspace,
                             size_t workspace_bytes, void* stream) {
-    int rc = attn_common_check(q, kcache, vcache, pos0, out, B, T, H, Hk, d, S_max, dtype);
+    int rc = lfw::attn_op_check(q, kcache, vcache, pos0, out, B, T, H, Hk, d, S_max, dtype);
     if (rc) return rc;
     if (!workspace) return fail(LLM_ERR_NULL_PTR, "workspace is NULL");
     // planned for keys up to the cache length; the workspace size (any length) covers it
@@ -1226,4 +1254,45 @@ int llm_op_attention_decode(const void* q, const void* kcache, const void* vcach
     return LLM_OK;
 }
 
+int llm_op_attention_decode_cluster(const void* q, const void* kcache, const void* vcache, const int32_t* pos0,
+                                    void* out, int B, int H, int Hk, int S_max, void* stream) {
+    int rc = lfw::attn_op_check(q, kcache, vcache, pos0, out, B, 1, H, Hk, 128, S_max, LLM_BF16);
+    if (rc) return rc;
+    const int cs = attn_cluster_size(B, H, Hk, 128, num_sms_current());
+    if (cs < 1) return fail(LLM_ERR_UNSUPPORTED, "cluster attention needs at most 8 query heads per KV head");
+    CUtensorMap tk, tv;
+    const uint64_t rows = (uint64_t)B * Hk * S_max;
+    if (!make_tmap(&tk, kcache, 128, rows, 64, 32) || !make_tmap(&tv, vcache, 128, rows, 64, 32))
+        return fail(LLM_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+    AttnClusterArgs a;
+    a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+    a.out = reinterpret_cast<__nv_bfloat16*>(out);
+    a.pos0 = pos0;
+    a.B = B;
+    a.H = H;
+    a.Hk = Hk;
+    a.S_max = S_max;
+    a.row_base = 0;
+    a.rows_per_seq = (long long)Hk * S_max;
+    a.cs = cs;
+    a.scale_log2 = (float)(1.4426950408889634 / sqrt(128.0));
+    a.err = op_err_ptr();
+    CK(launch_attn_cluster(a, &tk, &tv, reinterpret_cast<cudaStream_t>(stream)));
+    return LLM_OK;
+}
+
 }  // extern "C"
+
+// ---------------------------------------------------------------- shared with attn_decode_static.cu
+uint32_t* lfw::op_err_word() { return op_err_ptr(); }
+
+int lfw::attn_op_check(const void* q, const void* kc, const void* vc, const int32_t* pos0, const void* out, int B,
+                       int T, int H, int Hk, int d, int S_max, int dtype) {
+    if (!q || !kc || !vc || !pos0 || !out) return fail(LLM_ERR_NULL_PTR, "NULL operand");
+    if (B < 1 || T < 1 || H < 1 || Hk < 1 || H % Hk != 0 || S_max < 1 || d < 8 || d % 8 != 0 || d > 128)
+        return fail(LLM_ERR_BAD_ARG, "bad attention shape");
+    if (dtype != LLM_F32 && dtype != LLM_BF16) return fail(LLM_ERR_BAD_ARG, "bad dtype");
+    if (!aligned16(q) || !aligned16(kc) || !aligned16(vc) || !aligned16(out))
+        return fail(LLM_ERR_BAD_ARG, "operands must be 16-byte aligned");
+    return LLM_OK;
+}

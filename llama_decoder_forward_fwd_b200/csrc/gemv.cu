@@ -59,17 +59,22 @@ DEVI void logits_finish(const Epi& e, int M, int ntiles, int* last_s) {
 // cooperative (every CTA resident), so a row tile split over several CTAs is
 // finished by its first CTA, which waits for the other CTAs' pieces; they publish
 // them as soon as they reach the end of their part and move on.
-constexpr int GV_STAGES = 5;                    // ~110 KB per CTA: two CTAs (of consecutive
-                                                // launches) can share an SM
+// Ring depth: 5 stages (~110 KB per CTA) for the layer projections; the lm_head,
+// one long stream of 1 GB, keeps 10 stages in flight (measured: 163 against
+// 172 us at the Llama-3-8B vocabulary), which the layer projections do not gain from.
+template <int EPI> constexpr int gv_stages() { return EPI == EPI_LOGITS ? 10 : 5; }
 constexpr int GV_THREADS = GV_CONSUMERS + 32;   // 8 consumer warps + 1 producer warp
 constexpr int GV_XS_BYTES = 28 * 1024 + 256;    // token rows staged whole when they fit
-constexpr int GV_SMEM = 1024 + GV_STAGES * GV_UNIT_BYTES + GV_XS_BYTES + 2 * GV_STAGES * 8 + 64;
+template <int EPI> constexpr int gv_smem() {
+    return 1024 + gv_stages<EPI>() * GV_UNIT_BYTES + GV_XS_BYTES + 2 * gv_stages<EPI>() * 8 + 64;
+}
 
 template <int NB, int EPI>
-__global__ void __launch_bounds__(GV_THREADS, 2)
+__global__ void __launch_bounds__(GV_THREADS, gv_stages<EPI>() > 6 ? 1 : 2)
     gemv_bf16_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
                      const __grid_constant__ CUtensorMap tm2, const GemvArgs<__nv_bfloat16> a, int ntiles, int nku,
                      int max_pieces) {
+    constexpr int GV_STAGES = gv_stages<EPI>();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem + GV_STAGES * GV_UNIT_BYTES);
@@ -113,7 +118,8 @@ __global__ void __launch_bounds__(GV_THREADS, 2)
     X.K = a.K;
     X.Kp = nku * GV_BK;
     X.xs = (long long)a.M * X.Kp * 2 <= GV_XS_BYTES ? xs : nullptr;
-    gv_prologue(const_cast<__nv_bfloat16*>(X.xs), a.x, a.ldx, a.M, a.K, X.Kp, a.epi.norm, a.m0, rinv_s, rred_s);
+    gv_prologue(const_cast<__nv_bfloat16*>(X.xs), a.x, a.ldx, a.M, a.K, X.Kp, a.epi.norm, a.m0, rinv_s, rred_s, w.u0,
+                w.u1, nku);
     gv_consume<NB, EPI>(ring, w, X, a.N, a.m0, rinv_s, a.epi, a.ws, max_pieces, a.epi.err, DERR_GEMV_CONSUMER_WAIT);
 }
 
@@ -248,7 +254,7 @@ template <int NB, int EPI>
 static cudaError_t launch_bf16_e(const GemvArgs<__nv_bfloat16>& a, cudaStream_t s, bool pdl) {
     static bool smem_set = false;
     if (!smem_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_bf16_kernel<NB, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, GV_SMEM);
+        cudaError_t e = cudaFuncSetAttribute(gemv_bf16_kernel<NB, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv_smem<EPI>());
         if (e != cudaSuccess) return e;
         smem_set = true;
     }
@@ -263,7 +269,7 @@ static cudaError_t launch_bf16_e(const GemvArgs<__nv_bfloat16>& a, cudaStream_t 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid);
     cfg.blockDim = dim3(GV_THREADS);
-    cfg.dynamicSmemBytes = GV_SMEM;
+    cfg.dynamicSmemBytes = gv_smem<EPI>();
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;

@@ -168,9 +168,20 @@ DEVI void gv_drain(const GvRing& r, long long issued, uint32_t* err, uint32_t co
 // sums of h^2 left by the producer of the input (1 where the input is not
 // normed). Every load of the first batch is issued before any is used, so the
 // prologue costs about one memory round trip. Ends with a barrier of the consumers.
+// With a unit range [u0, u1) given (nku units per tile), only the 64-wide k
+// blocks those units read are copied: every CTA of a launch reads its own few
+// blocks instead of all of them reading the whole rows at once.
 DEVI void gv_prologue(__nv_bfloat16* xs, const __nv_bfloat16* x, int ldx, int M, int K, int Kp, const NormIn& n,
-                      int m0, float* rinv_s, float (*rred_s)[16]) {
+                      int m0, float* rinv_s, float (*rred_s)[16], long long u0 = 0, long long u1 = -1, int nku = 1) {
     constexpr int XB = 8;  // 16-byte loads per thread per batch
+    // k blocks [kb0, kb1] (inclusive, wrapping past the row's end) of the range, or all
+    const bool all_k = u1 < 0 || u1 - u0 >= nku;
+    const int kb0 = all_k ? 0 : (int)(u0 % nku), kb1 = all_k ? 0 : (int)((u1 - 1) % nku);
+    auto needed = [&](int k) {
+        if (all_k) return true;
+        const int kb = k / GV_BK;
+        return kb0 <= kb1 ? (kb >= kb0 && kb <= kb1) : (kb >= kb0 || kb <= kb1);
+    };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // partial sums: the first part of each row, loads only
     float part[16];
@@ -190,7 +201,7 @@ DEVI void gv_prologue(__nv_bfloat16* xs, const __nv_bfloat16* x, int ldx, int M,
                 v[j] = make_uint4(0, 0, 0, 0);
                 if (i < total) {
                     const int m = i / Kp, k = i - m * Kp;
-                    if (k < K) v[j] = __ldcg(reinterpret_cast<const uint4*>(x + (size_t)m * ldx + k));
+                    if (k < K && needed(k)) v[j] = __ldcg(reinterpret_cast<const uint4*>(x + (size_t)m * ldx + k));
                 }
             }
 #pragma unroll

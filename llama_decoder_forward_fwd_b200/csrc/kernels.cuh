@@ -171,6 +171,26 @@ struct AttnDecodePlan {
 AttnDecodePlan attn_decode_plan(int B, int T, int H, int Hk, int d, int max_keys, int num_sms);
 cudaError_t launch_attn_decode(const AttnDecodeArgs& a, bool bf16, cudaStream_t s, bool pdl);
 
+// Decode attention of one new token per sequence on the tensor cores, one
+// thread-block cluster per (sequence, KV head) group (attn_cluster.cu): bf16,
+// head_dim 128, at most 8 query heads per KV head. Needs no global scratch.
+struct AttnClusterArgs {
+    const __nv_bfloat16* q = nullptr;  // [B][H*128]
+    __nv_bfloat16* out = nullptr;      // [B][H*128]
+    const int32_t* pos0 = nullptr;     // [B] position of the new token (cache length before it)
+    int B = 0, H = 0, Hk = 0, S_max = 0;
+    long long row_base = 0;            // cache row of (sequence 0, KV head 0, position 0) in the maps
+    long long rows_per_seq = 0;        // cache rows between consecutive sequences
+    int cs = 1;                        // CTAs per group (the cluster size, 1..8)
+    float scale_log2 = 0.f;
+    uint32_t* err = nullptr;
+};
+// CTAs per group for B sequences of Hk KV heads on num_sms SMs (0: shape not supported).
+int attn_cluster_size(int B, int H, int Hk, int d, int num_sms);
+// tmK, tmV: the K and V caches as [rows][128] bf16 with 32-row, 64-column boxes.
+cudaError_t launch_attn_cluster(const AttnClusterArgs& a, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                cudaStream_t s);
+
 // ---- fused decode step (bf16): the whole model in one persistent launch ----
 struct DecodeStepArgs {
     int B = 0, D = 0, H = 0, Hk = 0, d = 0, F = 0, vocab = 0, S_max = 0, n_layers = 0;
@@ -243,6 +263,14 @@ cudaError_t launch_rope_tables(float* cosv, float* sinv, int n_pos, int half, do
 
 // Record msg as the calling thread's last error (llm_last_error) and return code.
 int set_error(int code, const char* msg);
+
+// Shared by the single-operation attention entry points: argument checks of the
+// split-KV and flash attention calls (0 or an LLM_ERR_* code, recorded), the
+// device error word their kernels report into, and the current device's SM count.
+int attn_op_check(const void* q, const void* kc, const void* vc, const int32_t* pos0, const void* out, int B, int T,
+                  int H, int Hk, int d, int S_max, int dtype);
+uint32_t* op_err_word();
+int current_num_sms();
 
 // Launch helper: programmatic stream serialization when pdl is set.
 template <typename... KArgs, typename... Args>

@@ -115,3 +115,39 @@ def test_split_kv_attention_matches_oracle(lib, dtype, d, tol, B, T, H, Hk, pos0
     torch.cuda.synchronize()
     err = np.abs(O.f64(out.cpu()) - ref)
     assert err.max() <= tol * float(vc.abs().max()), err.max()
+
+
+@pytest.mark.parametrize("B,H,Hk,S,pos0", [
+    (1, 32, 8, 2304, [2048]),          # the benchmark's decode: 8 groups, 8 CTAs per cluster
+    (1, 32, 8, 2304, [0]),             # a single key
+    (1, 32, 8, 2304, [2303]),          # the last position of the cache
+    (3, 32, 8, 1024, [31, 32, 700]),   # unit boundaries
+    (16, 32, 8, 8320, [4096, 8191, 5000, 6001, 4097, 7777, 8000, 4500, 6500, 7000, 5555, 4444, 8190, 6666, 5432, 7890]),
+    (8, 32, 32, 1152, [1024 + i for i in range(8)]),   # multi-head attention: one query head per KV head
+    (2, 16, 2, 512, [100, 3]),         # 8 query heads per KV head
+    (2, 12, 4, 300, [299, 150]),       # 3 query heads per KV head, a cache of 300 positions
+])
+def test_cluster_decode_attention_matches_oracle(lib, B, H, Hk, S, pos0):
+    """The tensor-core decode attention (one cluster per KV-head group, pieces merged
+    in distributed shared memory) against the oracle: the probabilities enter P V in
+    bf16 and the output is rounded to bf16, as in the flash kernel."""
+    import llama_decoder_forward_fwd_b200 as L
+    d = 128
+    q, kc, vc, ref = _attn_case(B, 1, H, Hk, d, S, pos0, torch.bfloat16, 31)
+    out = torch.full((B, 1, H * d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    p = torch.tensor(pos0, dtype=torch.int32, device=DEV)
+    for _ in range(2):
+        L.llm_op_attention_decode_cluster(q.to(DEV), kc.to(DEV), vc.to(DEV), p, out)
+    torch.cuda.synchronize()
+    err = np.abs(O.f64(out.cpu()) - ref)
+    assert err.max() <= 8e-3 * float(vc.abs().max()), err.max()
+
+
+def test_cluster_decode_attention_rejects_large_groups(lib):
+    import llama_decoder_forward_fwd_b200 as L
+    q = torch.zeros(1, 1, 32 * 128, dtype=torch.bfloat16, device=DEV)
+    kc = torch.zeros(1, 1, 64, 128, dtype=torch.bfloat16, device=DEV)
+    p = torch.zeros(1, dtype=torch.int32, device=DEV)
+    with pytest.raises(L.LlmError) as e:
+        L.llm_op_attention_decode_cluster(q.view(1, 1, 32, 128), kc, kc, p, q)
+    assert e.value.code == L.LLM_ERR_UNSUPPORTED
