@@ -118,6 +118,10 @@ struct llm_model {
     // activations and scratch
     float* h = nullptr;
     void *hw = nullptr, *q = nullptr, *o = nullptr, *g = nullptr;
+    // bf16 remainders of hw, o and g (split activations of the decode projections)
+    // and whether the last writer of each left them
+    void *hw_lo = nullptr, *o_lo = nullptr, *g_lo = nullptr;
+    bool hw_lo_ok = false, o_lo_ok = false, g_lo_ok = false;
     float* ss = nullptr;
     int ss_ld = 0;
     void *kc = nullptr, *vc = nullptr;
@@ -269,8 +273,17 @@ int project(llm_model* m, int l, int kind, int tkind, const void* x, const CUten
         ga.epi = epi;
         CK(launch_gemm_tc(ga, m->stream, m->pdl));
         if (nparts_out) *nparts_out = c.dim / GEMM_BN;
+        if (kind == EPI_RESID) m->hw_lo_ok = false;
+        if (kind == EPI_SWIGLU) m->g_lo_ok = false;
         return LLM_OK;
     }
+    // the input's remainders, when its producer left them
+    const void* x_lo = x == m->hw ? (m->hw_lo_ok ? m->hw_lo : nullptr)
+                     : x == m->o  ? (m->o_lo_ok ? m->o_lo : nullptr)
+                     : x == m->g  ? (m->g_lo_ok ? m->g_lo : nullptr) : nullptr;
+    Epi ep = epi;
+    if (m->bf16 && kind == EPI_RESID) ep.hw_lo_out = m->hw_lo;
+    if (m->bf16 && kind == EPI_SWIGLU) ep.g_lo_out = m->g_lo;
     for (int r0 = 0; r0 < M; r0 += 16) {
         const int rows = M - r0 < 16 ? M - r0 : 16;
         if (m->bf16) {
@@ -286,12 +299,13 @@ int project(llm_model* m, int l, int kind, int tkind, const void* x, const CUten
             ga.N = N;
             ga.K = K;
             ga.x = reinterpret_cast<const __nv_bfloat16*>(x) + (size_t)r0 * K;
+            ga.x_lo = x_lo ? reinterpret_cast<const __nv_bfloat16*>(x_lo) + (size_t)r0 * K : nullptr;
             ga.ldx = K;
             ga.M = rows;
             ga.m0 = r0;
             ga.num_sms = m->num_sms;
             ga.ws = m->gws;
-            ga.epi = epi;
+            ga.epi = ep;
             CK(launch_gemv_bf16(ga, m->stream, m->pdl));
         } else {
             GemvArgs<float> ga;
@@ -308,6 +322,8 @@ int project(llm_model* m, int l, int kind, int tkind, const void* x, const CUten
         }
     }
     if (nparts_out) *nparts_out = m->bf16 ? bf16_gemv_ss_parts(N) : f32_gemv_ss_parts(N);
+    if (kind == EPI_RESID) m->hw_lo_ok = m->bf16;
+    if (kind == EPI_SWIGLU) m->g_lo_ok = m->bf16;
     return LLM_OK;
 }
 
@@ -371,6 +387,7 @@ int run_phase(llm_model* m, int l, int p, int B, int T, int max_keys, int* npart
                 a.scale_log2 = scale_log2;
                 a.err = m->d_err;
                 CK(launch_attn_prefill(a, m->stream, m->pdl));
+                m->o_lo_ok = false;
             } else if (T == 1 && m->bf16 && m->kv32_ok && attn_cluster_size(B, H, Hk, d, m->num_sms) > 0) {
                 AttnClusterArgs a;
                 a.q = reinterpret_cast<const __nv_bfloat16*>(m->q);
@@ -382,10 +399,12 @@ int run_phase(llm_model* m, int l, int p, int B, int T, int max_keys, int* npart
                 a.S_max = c.max_seq_len;
                 a.row_base = (long long)l * c.max_batch * Hk * c.max_seq_len;
                 a.rows_per_seq = (long long)Hk * c.max_seq_len;
+                a.out_lo = reinterpret_cast<__nv_bfloat16*>(m->o_lo);
                 a.cs = attn_cluster_size(B, H, Hk, d, m->num_sms);
                 a.scale_log2 = scale_log2;
                 a.err = m->d_err;
                 CK(launch_attn_cluster(a, &m->tm_k32, &m->tm_v32, m->stream));
+                m->o_lo_ok = true;
             } else {
                 const AttnDecodePlan pl = attn_decode_plan(B, T, H, Hk, d, max_keys, m->num_sms);
                 if (pl.part_floats > m->attn_ws_floats || pl.counters > m->attn_cnt_n)
@@ -410,6 +429,7 @@ int run_phase(llm_model* m, int l, int p, int B, int T, int max_keys, int* npart
                 a.scale_log2 = scale_log2;
                 a.err = m->d_err;
                 CK(launch_attn_decode(a, m->bf16, m->stream, m->pdl));
+                m->o_lo_ok = false;
             }
             return LLM_OK;
         }
@@ -495,6 +515,7 @@ int run_head(llm_model* m, int B, int T, int nparts, int32_t* next, float* logit
         ga.N = c.vocab;
         ga.K = c.dim;
         ga.x = reinterpret_cast<const __nv_bfloat16*>(m->hw) + (size_t)(T - 1) * c.dim;
+        ga.x_lo = m->hw_lo_ok ? reinterpret_cast<const __nv_bfloat16*>(m->hw_lo) + (size_t)(T - 1) * c.dim : nullptr;
         ga.ldx = T * c.dim;
         ga.M = B;
         ga.num_sms = m->num_sms;
@@ -546,6 +567,8 @@ int run_embed(llm_model* m, const int32_t* tok, const float* h_in, int M) {
     ea.h_in = h_in;
     ea.h = m->h;
     ea.hw = m->hw;
+    ea.hw_lo = m->hw_lo;  // null for fp32 models
+    m->hw_lo_ok = m->bf16;
     ea.wnorm = m->L[0].attn_norm;
     ea.ss = m->ss;
     ea.M = M;
@@ -630,6 +653,7 @@ int run_fused_step(llm_model* m, int B, const int32_t* tok, const float* h_in, f
     KTimer timer(m, LLM_K_STEP);
     CK(cudaMemsetAsync(m->ds_bar, 0, 4, m->stream));
     CK(launch_decode_step(a, p, m->stream));
+    m->hw_lo_ok = m->o_lo_ok = m->g_lo_ok = false;
     return LLM_OK;
 }
 
@@ -730,6 +754,11 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
     MALLOC_OR_BAIL(m->q, Mx * H * d * es);
     MALLOC_OR_BAIL(m->o, Mx * H * d * es);
     MALLOC_OR_BAIL(m->g, Mx * F * es);
+    if (m->bf16) {
+        MALLOC_OR_BAIL(m->hw_lo, Mx * D * es);
+        MALLOC_OR_BAIL(m->o_lo, Mx * H * d * es);
+        MALLOC_OR_BAIL(m->g_lo, Mx * F * es);
+    }
     m->ss_ld = (int)Mx;
     const int parts = (bf16_gemv_ss_parts(D) > f32_gemv_ss_parts(D) ? bf16_gemv_ss_parts(D) : f32_gemv_ss_parts(D)) + 8;
     MALLOC_OR_BAIL(m->ss, (size_t)parts * Mx * 4);

@@ -57,6 +57,23 @@ DEVI float4 ld_dsmem_f32x4(uint32_t addr) {
     return v;
 }
 
+// Four output dims at element offset off: O / L in bf16, and the bf16 remainder
+// (split activations for the next projection) when asked.
+DEVI void attn_out4(const AttnClusterArgs& a, int off, const float (&O)[4], float L) {
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    const float v[4] = {O[0] * inv, O[1] * inv, O[2] * inv, O[3] * inv};
+    uint2 u;
+    u.x = pack_bf16x2(v[0], v[1]);
+    u.y = pack_bf16x2(v[2], v[3]);
+    *reinterpret_cast<uint2*>(a.out + off) = u;
+    if (a.out_lo) {
+        uint2 r;
+        r.x = pack_bf16x2(v[0] - bf16lo(u.x), v[1] - bf16hi(u.x));
+        r.y = pack_bf16x2(v[2] - bf16lo(u.y), v[3] - bf16hi(u.y));
+        *reinterpret_cast<uint2*>(a.out_lo + off) = r;
+    }
+}
+
 __global__ void __launch_bounds__(AC_THREADS, 1)
     attn_cluster_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const AttnClusterArgs a) {
@@ -130,11 +147,7 @@ __global__ void __launch_bounds__(AC_THREADS, 1)
             float M, L, O[4];
             attn_merge_warps<AC_CONSUMERS / 32>(wst, R, r, d4, M, L, O);
             if (a.cs == 1) {
-                const float inv = L > 0.f ? 1.f / L : 0.f;
-                uint2 u;
-                u.x = pack_bf16x2(O[0] * inv, O[1] * inv);
-                u.y = pack_bf16x2(O[2] * inv, O[3] * inv);
-                *reinterpret_cast<uint2*>(a.out + (size_t)b * a.H * 128 + (size_t)(kvh * R + r) * 128 + d4) = u;
+                attn_out4(a, b * a.H * 128 + (kvh * R + r) * 128 + d4, O, L);
             } else {
                 float* pr = piece + r * AW_REC;
                 *reinterpret_cast<float4*>(pr + 4 + d4) = make_float4(O[0], O[1], O[2], O[3]);
@@ -168,11 +181,7 @@ __global__ void __launch_bounds__(AC_THREADS, 1)
             if (q >= a.cs) break;
             lse_merge(M, L, O, mp[q], lp[q], op[q]);
         }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        uint2 u;
-        u.x = pack_bf16x2(O[0] * inv, O[1] * inv);
-        u.y = pack_bf16x2(O[2] * inv, O[3] * inv);
-        *reinterpret_cast<uint2*>(a.out + (size_t)b * a.H * 128 + (size_t)(kvh * R + r) * 128 + d4) = u;
+        attn_out4(a, b * a.H * 128 + (kvh * R + r) * 128 + d4, O, L);
     }
     cluster_sync_all();  // every piece stays in place until the first CTA has read it
 }

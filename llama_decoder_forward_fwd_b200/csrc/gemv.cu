@@ -59,17 +59,18 @@ DEVI void logits_finish(const Epi& e, int M, int ntiles, int* last_s) {
 // cooperative (every CTA resident), so a row tile split over several CTAs is
 // finished by its first CTA, which waits for the other CTAs' pieces; they publish
 // them as soon as they reach the end of their part and move on.
-// Ring depth: 5 stages (~110 KB per CTA) for the layer projections; the lm_head,
+// Ring depth: 5 stages for the layer projections; the lm_head,
 // one long stream of 1 GB, keeps 10 stages in flight (measured: 163 against
 // 172 us at the Llama-3-8B vocabulary), which the layer projections do not gain from.
 template <int EPI> constexpr int gv_stages() { return EPI == EPI_LOGITS ? 10 : 5; }
 constexpr int GV_THREADS = GV_CONSUMERS + 32;   // 8 consumer warps + 1 producer warp
-constexpr int GV_XS_BYTES = 28 * 1024 + 256;    // token rows staged whole when they fit
+constexpr int GV_XS_BYTES = 56 * 1024 + 256;    // token rows staged whole when they fit (one token's
+                                                // split rows of the 14336-wide FFN input)
 template <int EPI> constexpr int gv_smem() {
     return 1024 + gv_stages<EPI>() * GV_UNIT_BYTES + GV_XS_BYTES + 2 * gv_stages<EPI>() * 8 + 64;
 }
 
-template <int NB, int EPI>
+template <int NB, int EPI, bool SPLIT>
 __global__ void __launch_bounds__(GV_THREADS, gv_stages<EPI>() > 6 ? 1 : 2)
     gemv_bf16_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
                      const __grid_constant__ CUtensorMap tm2, const GemvArgs<__nv_bfloat16> a, int ntiles, int nku,
@@ -117,10 +118,13 @@ __global__ void __launch_bounds__(GV_THREADS, gv_stages<EPI>() > 6 ? 1 : 2)
     X.M = a.M;
     X.K = a.K;
     X.Kp = nku * GV_BK;
-    X.xs = (long long)a.M * X.Kp * 2 <= GV_XS_BYTES ? xs : nullptr;
+    X.xlo = SPLIT ? a.x_lo : nullptr;
+    X.MX = SPLIT ? 2 * a.M : a.M;
+    X.xs = (long long)X.MX * X.Kp * 2 <= GV_XS_BYTES ? xs : nullptr;
     gv_prologue(const_cast<__nv_bfloat16*>(X.xs), a.x, a.ldx, a.M, a.K, X.Kp, a.epi.norm, a.m0, rinv_s, rred_s, w.u0,
-                w.u1, nku);
-    gv_consume<NB, EPI>(ring, w, X, a.N, a.m0, rinv_s, a.epi, a.ws, max_pieces, a.epi.err, DERR_GEMV_CONSUMER_WAIT);
+                w.u1, nku, X.xlo);
+    gv_consume<NB, EPI, SPLIT>(ring, w, X, a.N, a.m0, rinv_s, a.epi, a.ws, max_pieces, a.epi.err,
+                               DERR_GEMV_CONSUMER_WAIT);
 }
 
 // fp32 kernel (CUDA cores): a warp owns a pair of logical rows, a CTA 8 pairs.
@@ -250,11 +254,12 @@ __global__ void __launch_bounds__(GEMV_THREADS) gemv_f32_kernel(const GemvArgs<f
 }
 
 // ---------------------------------------------------------------- launchers
-template <int NB, int EPI>
+template <int NB, int EPI, bool SPLIT>
 static cudaError_t launch_bf16_e(const GemvArgs<__nv_bfloat16>& a, cudaStream_t s, bool pdl) {
     static bool smem_set = false;
     if (!smem_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_bf16_kernel<NB, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, gv_smem<EPI>());
+        cudaError_t e = cudaFuncSetAttribute(gemv_bf16_kernel<NB, EPI, SPLIT>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, gv_smem<EPI>());
         if (e != cudaSuccess) return e;
         smem_set = true;
     }
@@ -278,17 +283,17 @@ static cudaError_t launch_bf16_e(const GemvArgs<__nv_bfloat16>& a, cudaStream_t 
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, gemv_bf16_kernel<NB, EPI>, m0, m1, m2, a, p.ntiles, p.nkb, p.max_pieces);
+    return cudaLaunchKernelEx(&cfg, gemv_bf16_kernel<NB, EPI, SPLIT>, m0, m1, m2, a, p.ntiles, p.nkb, p.max_pieces);
 }
 
-template <int NB>
+template <int NB, bool SPLIT>
 static cudaError_t launch_bf16_nb(const GemvArgs<__nv_bfloat16>& a, cudaStream_t s, bool pdl) {
     switch (a.epi.kind) {
-        case EPI_STORE_F32: return launch_bf16_e<NB, EPI_STORE_F32>(a, s, pdl);
-        case EPI_QKV_ROPE: return launch_bf16_e<NB, EPI_QKV_ROPE>(a, s, pdl);
-        case EPI_SWIGLU: return launch_bf16_e<NB, EPI_SWIGLU>(a, s, pdl);
-        case EPI_RESID: return launch_bf16_e<NB, EPI_RESID>(a, s, pdl);
-        case EPI_LOGITS: return launch_bf16_e<NB, EPI_LOGITS>(a, s, pdl);
+        case EPI_STORE_F32: return launch_bf16_e<NB, EPI_STORE_F32, SPLIT>(a, s, pdl);
+        case EPI_QKV_ROPE: return launch_bf16_e<NB, EPI_QKV_ROPE, SPLIT>(a, s, pdl);
+        case EPI_SWIGLU: return launch_bf16_e<NB, EPI_SWIGLU, SPLIT>(a, s, pdl);
+        case EPI_RESID: return launch_bf16_e<NB, EPI_RESID, SPLIT>(a, s, pdl);
+        case EPI_LOGITS: return launch_bf16_e<NB, EPI_LOGITS, SPLIT>(a, s, pdl);
     }
     return cudaErrorInvalidValue;
 }
@@ -324,7 +329,9 @@ size_t gemv_scratch_floats(int kind, int N, int K, int num_sms) {
 
 cudaError_t launch_gemv_bf16(const GemvArgs<__nv_bfloat16>& a, cudaStream_t s, bool pdl) {
     if (a.M < 1 || a.M > 16 || a.K % 8 != 0) return cudaErrorInvalidValue;
-    return a.M <= 8 ? launch_bf16_nb<8>(a, s, pdl) : launch_bf16_nb<16>(a, s, pdl);
+    if (a.x_lo && a.M <= 8)  // split activations: 2M B-operand columns
+        return a.M <= 4 ? launch_bf16_nb<8, true>(a, s, pdl) : launch_bf16_nb<16, true>(a, s, pdl);
+    return a.M <= 8 ? launch_bf16_nb<8, false>(a, s, pdl) : launch_bf16_nb<16, false>(a, s, pdl);
 }
 
 cudaError_t launch_gemv_f32(const GemvArgs<float>& a, cudaStream_t s, bool pdl) {

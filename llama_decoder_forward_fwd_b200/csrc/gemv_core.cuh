@@ -31,6 +31,14 @@
 //
 // Activations written earlier in the same launch by other CTAs (x, h, the
 // RMSNorm partial sums) are read with ld.global.cg (L2, never a stale L1 line).
+//
+// Split activations (SPLIT): in decode the producer of x also leaves its bf16
+// rounding remainder x_lo = bf16(x - bf16(x)). The B operand then holds 2M
+// columns, token m's bf16 part in column 2m and its remainder in column 2m + 1,
+// and the epilogue adds the two columns: the product sees x to about 16
+// significant bits instead of 8. A matrix-vector product is bound by its weight
+// bytes, and the extra columns fit in the MMA tile the tokens already occupy
+// (M <= 4) or in a second one (M <= 8), so the weight stream is unchanged.
 #pragma once
 #include "epilogue.cuh"
 
@@ -172,7 +180,8 @@ DEVI void gv_drain(const GvRing& r, long long issued, uint32_t* err, uint32_t co
 // blocks those units read are copied: every CTA of a launch reads its own few
 // blocks instead of all of them reading the whole rows at once.
 DEVI void gv_prologue(__nv_bfloat16* xs, const __nv_bfloat16* x, int ldx, int M, int K, int Kp, const NormIn& n,
-                      int m0, float* rinv_s, float (*rred_s)[16], long long u0 = 0, long long u1 = -1, int nku = 1) {
+                      int m0, float* rinv_s, float (*rred_s)[16], long long u0 = 0, long long u1 = -1, int nku = 1,
+                      const __nv_bfloat16* xlo = nullptr) {
     constexpr int XB = 8;  // 16-byte loads per thread per batch
     // k blocks [kb0, kb1] (inclusive, wrapping past the row's end) of the range, or all
     const bool all_k = u1 < 0 || u1 - u0 >= nku;
@@ -192,7 +201,7 @@ DEVI void gv_prologue(__nv_bfloat16* xs, const __nv_bfloat16* x, int ldx, int M,
                                   : 0.f;
     // token rows, XB loads in flight per thread
     if (xs != nullptr) {
-        const int total = M * Kp;
+        const int total = (xlo ? 2 * M : M) * Kp;  // with xlo: row 2m = x[m], row 2m + 1 = xlo[m]
         for (int i0 = threadIdx.x * 8; i0 < total; i0 += GV_CONSUMERS * 8 * XB) {
             uint4 v[XB];
 #pragma unroll
@@ -200,8 +209,9 @@ DEVI void gv_prologue(__nv_bfloat16* xs, const __nv_bfloat16* x, int ldx, int M,
                 const int i = i0 + j * GV_CONSUMERS * 8;
                 v[j] = make_uint4(0, 0, 0, 0);
                 if (i < total) {
-                    const int m = i / Kp, k = i - m * Kp;
-                    if (k < K && needed(k)) v[j] = __ldcg(reinterpret_cast<const uint4*>(x + (size_t)m * ldx + k));
+                    const int r = i / Kp, k = i - r * Kp;
+                    const __nv_bfloat16* src = xlo ? ((r & 1) ? xlo : x) + (size_t)(r >> 1) * ldx : x + (size_t)r * ldx;
+                    if (k < K && needed(k)) v[j] = __ldcg(reinterpret_cast<const uint4*>(src + k));
                 }
             }
 #pragma unroll
@@ -235,7 +245,9 @@ DEVI void gv_prologue(__nv_bfloat16* xs, const __nv_bfloat16* x, int ldx, int M,
 struct GvX {
     const __nv_bfloat16* x;  // [M][ldx] in global memory
     int ldx, M, K, Kp;       // Kp: K padded to the unit width (the TMA box fills zeros past K)
-    const __nv_bfloat16* xs; // [M][Kp] copy in shared memory, or nullptr
+    const __nv_bfloat16* xs; // [MX][Kp] copy in shared memory, or nullptr
+    const __nv_bfloat16* xlo = nullptr;  // split activations: the remainders, [M][ldx]
+    int MX = 0;                          // B-operand columns: M, or 2M when split
 };
 
 // Operands of a tile's epilogue that live in global memory: for the residual
@@ -251,7 +263,12 @@ struct GvEpiOps {
     float w[2];             // next norm weight of rows g / g+8
 };
 
-template <int NB, int EPI>
+// Token of accumulator column (n, h): 2t4 + h of n-tile n, or with split
+// activations the column pair (2t4, 2t4 + 1) of n-tile n, token n*4 + t4 (h = 0).
+template <bool SPLIT>
+DEVI int gv_token(int n, int h, int t4) { return SPLIT ? n * 4 + t4 : n * 8 + 2 * t4 + h; }
+
+template <int NB, int EPI, bool SPLIT = false>
 DEVI void gv_epi_prefetch(GvEpiOps<NB>& op, int tile, int N, int M, int m0, const Epi& e) {
     if (EPI != EPI_RESID && EPI != EPI_QKV_ROPE) return;
     constexpr int NM = NB / 8;
@@ -269,12 +286,13 @@ DEVI void gv_epi_prefetch(GvEpiOps<NB>& op, int tile, int N, int M, int m0, cons
     for (int n = 0; n < NM; ++n)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const int m = n * 8 + 2 * t4 + h;
+            const int m = gv_token<SPLIT>(n, h, t4);
             const int mg = m0 + m;
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 op.a[n][h][q] = 0.f;
                 op.b[n][h][q] = 0.f;
+                if (SPLIT && h == 1) continue;
                 if (m >= M || lr[q] >= N) continue;
                 if (EPI == EPI_RESID) {
                     op.a[n][h][q] = __ldcg(e.h + (long long)mg * e.D + lr[q]);
@@ -316,7 +334,7 @@ DEVI void gv_qkv_pair(const Epi& e, int m, int col, float v0, float v1, float cs
 
 // Fused epilogue of one warp's 16 rows of a finished row tile (accumulators c,
 // before the RMSNorm scale; global operands in op).
-template <int NB, int EPI>
+template <int NB, int EPI, bool SPLIT = false>
 DEVI void gv_epilogue(int tile, const float (&c)[NB / 8][4], int N, int M, int m0, const float* rinv_s, const Epi& e,
                       const GemvScratch& ws, int ntiles, const GvEpiOps<NB>& op) {
     constexpr int NM = NB / 8;
@@ -335,13 +353,14 @@ DEVI void gv_epilogue(int tile, const float (&c)[NB / 8][4], int N, int M, int m
     for (int n = 0; n < NM; ++n)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const int m = n * 8 + 2 * t4 + h;
+            const int m = gv_token<SPLIT>(n, h, t4);
             ssum[n][h] = 0.f;
             bv[n][h] = -FLT_MAX;
             bi[n][h] = INT_MAX;
+            if (SPLIT && h == 1) continue;  // (uniform over the warp)
             const float r = m < M ? rinv_s[m] : 0.f;
-            const float v0 = c[n][h] * r;      // A row g
-            const float v1 = c[n][2 + h] * r;  // A row g + 8
+            const float v0 = (SPLIT ? c[n][0] + c[n][1] : c[n][h]) * r;          // A row g
+            const float v1 = (SPLIT ? c[n][2] + c[n][3] : c[n][2 + h]) * r;      // A row g + 8
             if (EPI == EPI_QKV_ROPE) {
                 // RoPE pairs (2i, 2i+1) sit in A rows g and g^1: lanes lane and lane^4.
                 const float p0 = __shfl_xor_sync(0xffffffffu, v0, 4);
@@ -359,22 +378,30 @@ DEVI void gv_epilogue(int tile, const float (&c)[NB / 8][4], int N, int M, int m
                 if (lr0 >= 0) e.y[(size_t)mg * e.ldy + lr0] = v0;
                 if (lr1 >= 0) e.y[(size_t)mg * e.ldy + lr1] = v1;
             } else if (EPI == EPI_SWIGLU) {
-                if (lr0 >= 0)
-                    reinterpret_cast<__nv_bfloat16*>(e.g_out)[(size_t)mg * e.F + lr0] = __float2bfloat16_rn(swiglu(v0, v1));
+                if (lr0 >= 0) {
+                    const float gv = swiglu(v0, v1);
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(gv);
+                    reinterpret_cast<__nv_bfloat16*>(e.g_out)[(size_t)mg * e.F + lr0] = hi;
+                    if (e.g_lo_out)
+                        reinterpret_cast<__nv_bfloat16*>(e.g_lo_out)[(size_t)mg * e.F + lr0] =
+                            __float2bfloat16_rn(gv - __bfloat162float(hi));
+                }
             } else if (EPI == EPI_RESID) {
                 // residual add and the next norm's input hw = h * w (as epi_resid1,
-                // with h and w from the prefetch)
+                // with h and w from the prefetch), and its remainder when asked
                 float sq = 0.f;
-                if (lr0 >= 0) {
-                    const float hn = op.a[n][h][0] + v0;
-                    e.h[(long long)mg * e.D + lr0] = hn;
-                    reinterpret_cast<__nv_bfloat16*>(e.hw_out)[(long long)mg * e.D + lr0] = __float2bfloat16_rn(hn * op.w[0]);
-                    sq += hn * hn;
-                }
-                if (lr1 >= 0) {
-                    const float hn = op.a[n][h][1] + v1;
-                    e.h[(long long)mg * e.D + lr1] = hn;
-                    reinterpret_cast<__nv_bfloat16*>(e.hw_out)[(long long)mg * e.D + lr1] = __float2bfloat16_rn(hn * op.w[1]);
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int lr = q ? lr1 : lr0;
+                    if (lr < 0) continue;
+                    const float hn = op.a[n][h][q] + (q ? v1 : v0);
+                    e.h[(long long)mg * e.D + lr] = hn;
+                    const float xw = hn * op.w[q];
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(xw);
+                    reinterpret_cast<__nv_bfloat16*>(e.hw_out)[(long long)mg * e.D + lr] = hi;
+                    if (e.hw_lo_out)
+                        reinterpret_cast<__nv_bfloat16*>(e.hw_lo_out)[(long long)mg * e.D + lr] =
+                            __float2bfloat16_rn(xw - __bfloat162float(hi));
                     sq += hn * hn;
                 }
                 ssum[n][h] = sq;
@@ -394,6 +421,7 @@ DEVI void gv_epilogue(int tile, const float (&c)[NB / 8][4], int N, int M, int m
         for (int n = 0; n < NM; ++n)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
+                if (SPLIT && h == 1) continue;
 #pragma unroll
                 for (int o = 4; o < 32; o <<= 1) {  // over the 8 row groups g
                     if (EPI == EPI_RESID) {
@@ -404,7 +432,7 @@ DEVI void gv_epilogue(int tile, const float (&c)[NB / 8][4], int N, int M, int m
                         am_merge(bv[n][h], bi[n][h], ov, oi);
                     }
                 }
-                const int m = n * 8 + 2 * t4 + h;
+                const int m = gv_token<SPLIT>(n, h, t4);
                 if (g == 0 && m < M) {
                     if (EPI == EPI_RESID)  // one part per 16 rows
                         e.ss_out[(size_t)(tile * 8 + warp) * e.ss_out_ld + m0 + m] = ssum[n][h];
@@ -440,13 +468,14 @@ DEVI void gv_epilogue(int tile, const float (&c)[NB / 8][4], int N, int M, int m
 // tile reduction and the epilogues. A failed (timed-out) wait is recorded in
 // *err; the warp then stops waiting and runs the rest of its control flow on
 // whatever the stage holds, so every consumer warp still reaches every barrier.
-template <int NB, int EPI>
+template <int NB, int EPI, bool SPLIT = false>
 DEVI bool gv_consume(GvRing& r, const GvWork& w, const GvX& X, int N, int m0, const float* rinv_s, const Epi& e,
                      const GemvScratch& ws, int max_pieces, uint32_t* err, uint32_t code) {
     constexpr int NM = NB / 8;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t4 = lane & 3;
     const int M = X.M, K = X.K;
+    const int MX = SPLIT ? 2 * M : M;  // B-operand columns
     const long long G = w.G;
     bool ok = true;
     // this warp's two A rows (g and g + 8) inside a stage
@@ -461,7 +490,7 @@ DEVI bool gv_consume(GvRing& r, const GvWork& w, const GvX& X, int N, int m0, co
     GvEpiOps<NB> ops;
     for (long long u = w.u0; u < w.u1; ++u) {
         // this CTA holds the tile's first unit, so it runs the tile's epilogue
-        if (ckb == 0) gv_epi_prefetch<NB, EPI>(ops, ctile, N, M, m0, e);
+        if (ckb == 0) gv_epi_prefetch<NB, EPI, SPLIT>(ops, ctile, N, M, m0, e);
         if (ok && !mbar_wait(&r.full[r.st], r.ph, err, code)) ok = false;
         const uint32_t sp = smem_u32(r.stages + r.st * GV_UNIT_BYTES);
         const int kx = ckb * GV_BK;
@@ -482,14 +511,15 @@ DEVI bool gv_consume(GvRing& r, const GvWork& w, const GvX& X, int N, int m0, co
                 const uint32_t xp = xbase + (uint32_t)(mrow * X.Kp + k) * 2;
                 xa[n] = z4;
                 xb[n] = z4;
-                if (mrow < M) {
+                if (mrow < MX) {
                     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(xa[n].x), "=r"(xa[n].y), "=r"(xa[n].z), "=r"(xa[n].w) : "r"(xp));
                     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(xb[n].x), "=r"(xb[n].y), "=r"(xb[n].z), "=r"(xb[n].w) : "r"(xp + 16));
                 }
             } else {
-                const __nv_bfloat16* xp = X.x + (size_t)mrow * X.ldx + k;
-                xa[n] = (mrow < M && k < K) ? __ldcg(reinterpret_cast<const uint4*>(xp)) : z4;
-                xb[n] = (mrow < M && k + 8 < K) ? __ldcg(reinterpret_cast<const uint4*>(xp + 8)) : z4;
+                const __nv_bfloat16* xp = (SPLIT ? ((mrow & 1) ? X.xlo : X.x) + (size_t)(mrow >> 1) * X.ldx
+                                                 : X.x + (size_t)mrow * X.ldx) + k;
+                xa[n] = (mrow < MX && k < K) ? __ldcg(reinterpret_cast<const uint4*>(xp)) : z4;
+                xb[n] = (mrow < MX && k + 8 < K) ? __ldcg(reinterpret_cast<const uint4*>(xp + 8)) : z4;
             }
         }
         __syncwarp();
@@ -516,7 +546,7 @@ DEVI bool gv_consume(GvRing& r, const GvWork& w, const GvX& X, int N, int m0, co
         const long long tu0 = (long long)tile * w.nku;
         const long long cf = cta_of_unit(tu0, G, w.TU), cl = cta_of_unit(tu0 + w.nku - 1, G, w.TU);
         if (cf == cl) {
-            gv_epilogue<NB, EPI>(tile, c, N, M, m0, rinv_s, e, ws, w.ntiles, ops);
+            gv_epilogue<NB, EPI, SPLIT>(tile, c, N, M, m0, rinv_s, e, ws, w.ntiles, ops);
         } else {
             // Every CTA of the tile but the first publishes its piece, one warp's rows
             // at a time; the first CTA's warps wait for their rows' pieces.
@@ -560,7 +590,7 @@ DEVI bool gv_consume(GvRing& r, const GvWork& w, const GvX& X, int N, int m0, co
                         t[n][3] += v.w;
                     }
                 }
-                gv_epilogue<NB, EPI>(tile, t, N, M, m0, rinv_s, e, ws, w.ntiles, ops);
+                gv_epilogue<NB, EPI, SPLIT>(tile, t, N, M, m0, rinv_s, e, ws, w.ntiles, ops);
             }
         }
 #pragma unroll

@@ -55,11 +55,13 @@ struct Epi {
     void* v_cache = nullptr;
     // EPI_SWIGLU
     void* g_out = nullptr;
+    void* g_lo_out = nullptr;  // bf16 remainder of g (split activations; may be null)
     int F = 0;
     // EPI_RESID
     float* h = nullptr;
     int D = 0;
     void* hw_out = nullptr;
+    void* hw_lo_out = nullptr;  // bf16 remainder of hw (split activations; may be null)
     const void* wnext = nullptr;
     float* ss_out = nullptr;
     int ss_out_ld = 0;
@@ -107,6 +109,7 @@ struct GemvArgs {
     int N = 0;                                    // logical output rows (SWIGLU: ffn_hidden)
     int K = 0;
     const T* x = nullptr;  // [M][ldx]
+    const T* x_lo = nullptr;  // bf16 kernel, M <= 8: the bf16 remainders of x (split activations)
     int ldx = 0;
     int M = 0;   // rows in this launch (<= 16)
     int m0 = 0;  // token index of row 0 (the epilogue sees token m0 + m)
@@ -177,6 +180,7 @@ cudaError_t launch_attn_decode(const AttnDecodeArgs& a, bool bf16, cudaStream_t 
 struct AttnClusterArgs {
     const __nv_bfloat16* q = nullptr;  // [B][H*128]
     __nv_bfloat16* out = nullptr;      // [B][H*128]
+    __nv_bfloat16* out_lo = nullptr;   // [B][H*128] bf16 remainder of the output, or null
     const int32_t* pos0 = nullptr;     // [B] position of the new token (cache length before it)
     int B = 0, H = 0, Hk = 0, S_max = 0;
     long long row_base = 0;            // cache row of (sequence 0, KV head 0, position 0) in the maps
@@ -250,6 +254,7 @@ struct EmbedArgs {
     const float* h_in = nullptr;   // or given hidden states [M][D]
     float* h = nullptr;
     void* hw = nullptr;
+    void* hw_lo = nullptr;         // bf16 models: the remainder hw - bf16(hw), or null
     const void* wnorm = nullptr;   // first layer's attention_norm
     float* ss = nullptr;           // [1][M]
     int M = 0, D = 0, vocab = 0;

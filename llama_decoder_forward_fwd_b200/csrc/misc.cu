@@ -21,6 +21,7 @@ __global__ void __launch_bounds__(EMB_THREADS) embed_kernel(const EmbedArgs a) {
     pdl_wait();
     const WT* wn = reinterpret_cast<const WT*>(a.wnorm);
     WT* hw = reinterpret_cast<WT*>(a.hw) + (long long)m * a.D;
+    WT* hw_lo = a.hw_lo ? reinterpret_cast<WT*>(a.hw_lo) + (long long)m * a.D : nullptr;
     float* h = a.h + (long long)m * a.D;
     const WT* src = nullptr;
     const float* hsrc = nullptr;
@@ -48,7 +49,9 @@ __global__ void __launch_bounds__(EMB_THREADS) embed_kernel(const EmbedArgs a) {
         reinterpret_cast<float4*>(h + i)[1] = make_float4(v[4], v[5], v[6], v[7]);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            hw[i + j] = from_f<WT>(v[j] * w[j]);
+            const WT xw = from_f<WT>(v[j] * w[j]);
+            hw[i + j] = xw;
+            if (hw_lo) hw_lo[i + j] = from_f<WT>(v[j] * w[j] - to_f<WT>(xw));
             ss += v[j] * v[j];
         }
     }

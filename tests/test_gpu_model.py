@@ -186,6 +186,45 @@ def test_batched_decode_over_prefilled_ragged_caches(lib):
     model.free()
 
 
+def test_batched_decode_at_the_workload_cache_lengths(lib):
+    """The batched-decode workload at its own sizes (two Llama-3-8B layers): 16
+    sequences whose caches hold 4096-8192 N(0,1) positions, decoded through the
+    CUDA graph; per-layer hidden states, logits and argmax against the oracle
+    (which feeds its own tokens to both sides)."""
+    w = S.WORKLOADS["llama3-8b-bf16-b16-kv4k8k-g128"]
+    shape = w.shape.replace(n_layers=2)
+    B = w.batch
+    model, orc = build_pair(shape, w.seed, batch=B, max_tokens=B, flags=L.LLM_FLAG_CUDA_GRAPH)
+    lens, caches = S.make_kv_prefill(shape, w.seed, B, *w.kv_len_range)
+    assert int(lens.min()) >= 4096 and int(lens.max()) <= 8192
+    install_prefilled_cache(model, orc, lens.numpy(), caches)
+    del caches
+    tok = S.make_tokens(w.seed, B, 1, shape.vocab, tag="decode0")[:, 0].numpy()
+    nxt = torch.empty(B, dtype=torch.int32, device=DEV)
+    logits = torch.empty(B, shape.vocab, device=DEV)
+    checked = 0
+    for step in range(2):
+        L.llm_decode_step(model.h, torch.as_tensor(tok, dtype=torch.int32).to(DEV), nxt, logits)
+        L.llm_synchronize(model.h)
+        o_taps = []
+        tok, o_logits = orc.decode(tok, o_taps)
+        check_taps(gpu_taps(model, B), [t.reshape(B, -1) for t in o_taps], what=f"step {step}")
+        assert rel_l2(logits.cpu().numpy(), o_logits) <= BF16_REL_L2
+        checked += check_argmax(nxt.cpu().numpy(), o_logits)
+    assert L.llm_kv_cache_get_lens(model.h, B) == [int(x) + 2 for x in lens]
+    assert checked >= B
+    model.free()
+
+
+def test_llama2_mha_at_the_workload_batch_and_prompt(lib):
+    """The Llama-2-7B multi-head workload at its own batch and prompt length (two
+    layers): 8 sequences of 1024 tokens through the tensor-core prefill, then
+    decode steps; per-layer hidden states, logits and argmax against the oracle."""
+    w = S.WORKLOADS["llama2-7b-mha-bf16-b8-p1024-g256"]
+    shape = w.shape.replace(n_layers=2, max_seq_len=w.prompt_len + 8)
+    _run_tokens_case(shape, seed=w.seed, B=w.batch, T=w.prompt_len, steps=2, flags=L.LLM_FLAG_CUDA_GRAPH)
+
+
 def test_long_context_decode_up_to_the_8192_context(lib):
     """Batch-1 decode against a cache of 8064 positions (two Llama-3-8B layers):
     many 32-key groups per attention warp and the longest cache the context allows."""

@@ -151,3 +151,23 @@ def test_cluster_decode_attention_rejects_large_groups(lib):
     with pytest.raises(L.LlmError) as e:
         L.llm_op_attention_decode_cluster(q.view(1, 1, 32, 128), kc, kc, p, q)
     assert e.value.code == L.LLM_ERR_UNSUPPORTED
+
+
+def test_split_kv_attention_batch_16_long_caches_matches_oracle(lib):
+    """The split-KV kernel at the batched-decode workload's shape (16 sequences,
+    caches of 4096-8192 positions): the plan splits by length (12 splits of more
+    than 704 keys per CTA) rather than to fill the GPU."""
+    import llama_decoder_forward_fwd_b200 as L
+    import seeded_inputs as S
+    w = S.WORKLOADS["llama3-8b-bf16-b16-kv4k8k-g128"]
+    B, H, Hk, d, S_max = w.batch, 32, 8, 128, 8192
+    lens = S.make_kv_prefill(w.shape, w.seed, B, *w.kv_len_range, layers=[])[0]
+    pos0 = [min(int(x), S_max - 1) for x in lens]
+    q, kc, vc, ref = _attn_case(B, 1, H, Hk, d, S_max, pos0, torch.bfloat16, 41)
+    out = torch.full((B, 1, H * d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    p = torch.tensor(pos0, dtype=torch.int32, device=DEV)
+    ws = torch.empty(L.llm_op_attention_decode_workspace(B, 1, H, Hk, d), dtype=torch.uint8, device=DEV)
+    L.llm_op_attention_decode(q.to(DEV), kc.to(DEV), vc.to(DEV), p, out, ws)
+    torch.cuda.synchronize()
+    err = np.abs(O.f64(out.cpu()) - ref)
+    assert err.max() <= 6e-3 * float(vc.abs().max()), err.max()
