@@ -383,6 +383,12 @@ def run_ours(args, rank, world, local_rank):
     kernel_table = {k: {"ms": round(v[0], 3), "launches": v[1], "share": round(v[0] / tot, 4)}
                     for k, v in sorted(shares.items(), key=lambda kv: -kv[1][0])}
     model.free()
+    workloads = None
+    if world == 1 and not args.no_workloads:
+        # after the timed region: the headline weights go, each workload brings its own
+        del glob, layers, model, tm
+        torch.cuda.empty_cache()
+        workloads = workloads_block()
 
     if rank != 0:
         return
@@ -403,11 +409,44 @@ def run_ours(args, rank, world, local_rank):
                                       G * (1 if fused else 5 * shape.n_layers + 2)),
         "clocks": clocks,
     }
+    if workloads is not None:
+        line["workloads"] = workloads
     print(json.dumps(line), flush=True)
 
 
 # ---------------------------------------------------------------- the other workloads
 def run_workload(args):
+    """The --workload command: one JSON line for that workload."""
+    print(json.dumps(measure_workload(args.workload, args.steps, args.warmup, args.fused, args.no_graph)), flush=True)
+
+
+# the other workloads, summarised in the headline line (decode and prefill at each one's own sizes)
+OTHER_WORKLOADS = ("llama3-8b-bf16-b16-kv4k8k-g128", "llama2-7b-mha-bf16-b8-p1024-g256",
+                   "llama3-8b-bf16-b1-kv8k-g128", "llama3-8b-mqa-bf16-b1-p2048-g256")
+
+
+def workloads_block(steps=1, warmup=1):
+    """Compact decode (and prefill) numbers of OTHER_WORKLOADS, one pass each after a warm-up."""
+    import torch
+    out = {}
+    for name in OTHER_WORKLOADS:
+        d = measure_workload(name, steps, warmup, fused=False, no_graph=False, kernel_times=False)
+        rec = {"batch": d["config"]["batch"], "decode_steps": d["config"]["decode_steps"],
+               "decode_tok_s": round(d["decode"]["tok_s"], 1),
+               "decode_ms_per_step": round(d["decode"]["ms_per_step"], 4),
+               "decode_frac_of_hbm": round(d["decode"]["frac_of_hbm"], 4)}
+        if d["config"]["input"] == "kv_prefilled":
+            rec["cache_lengths"] = d["config"]["cache_lengths"]
+        if "prefill" in d:
+            rec["prompt_len"] = d["config"]["prompt_len"]
+            rec["prefill_tok_s"] = round(d["prefill"]["tok_s"], 1)
+            rec["prefill_frac_of_bf16_peak"] = round(d["prefill"]["frac_of_bf16_peak"], 4)
+        out[name] = rec
+        torch.cuda.empty_cache()
+    return out
+
+
+def measure_workload(name, steps, warmup, fused=False, no_graph=False, kernel_times=True):
     """Prefill and decode throughput of a workload other than the headline one (one GPU).
 
     Token workloads: a prefill of the prompt, then greedy decode steps (CUDA
@@ -421,15 +460,15 @@ def run_workload(args):
     import llama_decoder_forward_fwd_b200 as L
     import seeded_inputs as S
 
-    w = S.WORKLOADS[args.workload]
+    w = S.WORKLOADS[name]
     shape, B, T, G = w.shape, w.batch, w.prompt_len, w.decode_steps
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
     glob, layers = S.make_weights(shape, w.seed, device=dev)
     stream = torch.cuda.Stream(device=dev)
-    graph = w.input_kind != "hidden" and not args.no_graph
-    flags = (L.LLM_FLAG_CUDA_GRAPH if graph else 0) | (L.LLM_FLAG_FUSED_DECODE if args.fused else 0)
+    graph = w.input_kind != "hidden" and not no_graph
+    flags = (L.LLM_FLAG_CUDA_GRAPH if graph else 0) | (L.LLM_FLAG_FUSED_DECODE if fused else 0)
     mt = B * T if T else B
     model = L.Model(shape, glob, layers, max_batch=B, max_tokens=mt, flags=flags, stream=stream, device=dev)
     D, Hk, d, Ln = shape.dim, shape.n_kv_heads, shape.head_dim, shape.n_layers
@@ -466,13 +505,13 @@ def run_workload(args):
         kc.normal_()
         vc.normal_()
         torch.cuda.synchronize(dev)
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         prefill()
         decode()
     torch.cuda.synchronize(dev)
     pre_ms, dec_ms = [], []
     with ClockSampler(0) as clk:
-        for _ in range(args.steps):
+        for _ in range(steps):
             e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
             e0.record(stream)
             prefill()
@@ -484,21 +523,23 @@ def run_workload(args):
             dec_ms.append(e1.elapsed_time(e2))
     L.llm_synchronize(model.h)
     model.free()
-    # per-kernel decode time: a second pass with the library's CUDA-event timing
-    tm = L.Model(shape, model.glob, model.layers, max_batch=B, max_tokens=mt,
-                 flags=flags | L.LLM_FLAG_KERNEL_TIMING, stream=stream, device=dev)
-    model = tm
-    if w.input_kind == "kv_prefilled":
-        kc, vc = model.kv_cache_tensors()
-        kc.normal_()
-        vc.normal_()
-        torch.cuda.synchronize(dev)
-    for rep in range(2):  # the first pass captures the graphs
-        prefill()
-        L.llm_kernel_times(model.h, reset=True)
-        decode()
-        kt = L.llm_kernel_times(model.h, reset=True)
-    model.free()
+    kt = {}
+    if kernel_times:
+        # per-kernel decode time: a second pass with the library's CUDA-event timing
+        tm = L.Model(shape, model.glob, model.layers, max_batch=B, max_tokens=mt,
+                     flags=flags | L.LLM_FLAG_KERNEL_TIMING, stream=stream, device=dev)
+        model = tm
+        if w.input_kind == "kv_prefilled":
+            kc, vc = model.kv_cache_tensors()
+            kc.normal_()
+            vc.normal_()
+            torch.cuda.synchronize(dev)
+        for rep in range(2):  # the first pass captures the graphs
+            prefill()
+            L.llm_kernel_times(model.h, reset=True)
+            decode()
+            kt = L.llm_kernel_times(model.h, reset=True)
+        model.free()
     # algorithmic work: every weight once per decode step, each sequence's cache once
     head = shape.has_embed_and_head
     S_mean = sum(lens) / B + G / 2
@@ -513,10 +554,10 @@ def run_workload(args):
     step_bytes = esz * (lin_params + (shape.vocab * D if head else 0)) + Ln * B * 2 * Hk * d * esz * S_mean
     dec_s = statistics.median(dec_ms) / 1e3
     line = {"impl": "ours", "workload": w.name, "metric": "decode tokens/s; % of measured HBM (and prefill % of bf16 peak)",
-            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "dtype": shape.dtype, "data": "synthetic",
+            "n_gpus": 1, "steps": steps, "warmup": warmup, "dtype": shape.dtype, "data": "synthetic",
             "config": {"workload": w.name, "batch": B, "prompt_len": T, "decode_steps": G, "input": w.input_kind,
                        "cache_lengths": [min(lens), max(lens)], "cuda_graph_decode": graph,
-                       "decode_kernel": "fused step" if args.fused else "layerwise"},
+                       "decode_kernel": "fused step" if fused else "layerwise"},
             "decode": {"tok_s": B * G / dec_s, "ms_per_step": dec_s * 1e3 / G, "gbs": step_bytes * G / dec_s / 1e9,
                        "frac_of_hbm": step_bytes * G / dec_s / 1e9 / peaks["hbm_gbs"], "bytes_per_step": step_bytes,
                        "peak_gbs": peaks["hbm_gbs"], "peak_source": peak_src, "kernels": kernels},
@@ -528,7 +569,7 @@ def run_workload(args):
                                                  if shape.dtype == "bf16" else None)}
     line["value"] = line["decode"]["tok_s"]
     line["unit"] = "tokens/s"
-    print(json.dumps(line), flush=True)
+    return line
 
 
 def main():
@@ -539,6 +580,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="leave out the compact block of the other workloads' numbers (single GPU only)")
     ap.add_argument("--pdl", action="store_true",
                     help="programmatic dependent launch between consecutive kernels")
     ap.add_argument("--fused", action="store_true",

@@ -211,6 +211,21 @@ int llm_debug_tap(llm_model* m, int layer, float* dst, size_t dst_elems);
  */
 int llm_kernel_times(llm_model* m, int n, double* total_ms, int64_t* launches, int reset);
 
+/*
+ * Failure detection, exercised on purpose: queues on the model's stream a
+ * kernel that enters one of the library's bounded device waits with a target
+ * that is never reached, bounded by limit_ms (0 < limit_ms <= 10000) instead of
+ * the usual 4 s: which = 0 an mbarrier wait for bytes no copy delivers, which = 1
+ * a grid barrier of a two-CTA cooperative launch that waits for twice the
+ * arrivals its CTAs make.
+ * The wait gives up, records its code in the model's device error word and the
+ * kernel returns: nothing faults or hangs, and the next llm_synchronize()
+ * returns LLM_ERR_DEVICE_TIMEOUT (clearing the word) while the model stays
+ * usable. The pages have no counterpart: this is a diagnostic of the library.
+ * Returns LLM_OK once queued, LLM_ERR_BAD_ARG or LLM_ERR_CUDA otherwise.
+ */
+int llm_debug_wait_probe(llm_model* m, int which, double limit_ms);
+
 /* Wait for the model's stream; report a CUDA error or a device-side timeout. */
 int llm_synchronize(llm_model* m);
 

@@ -70,6 +70,7 @@ _SIGS = {
     "llm_kv_cache_get_lens": (_i, [_vp, ctypes.POINTER(ctypes.c_int32), _i]),
     "llm_debug_tap": (_i, [_vp, _i, _vp, _sz]),
     "llm_kernel_times": (_i, [_vp, _i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), _i]),
+    "llm_debug_wait_probe": (_i, [_vp, _i, ctypes.c_double]),
     "llm_synchronize": (_i, [_vp]),
     "llm_model_free": (None, [_vp]),
     "llm_last_error": (ctypes.c_char_p, []),
@@ -179,6 +180,11 @@ def llm_kernel_times(m, reset: bool = True):
     cnt = (ctypes.c_int64 * n)()
     check(load().llm_kernel_times(m, n, ms, cnt, int(reset)))
     return {k: (ms[i], cnt[i]) for i, k in enumerate(KERNEL_KINDS)}
+
+
+def llm_debug_wait_probe(m, which: int, limit_ms: float):
+    """Queue a bounded device wait that cannot complete (0: mbarrier, 1: grid barrier)."""
+    check(load().llm_debug_wait_probe(m, which, float(limit_ms)))
 
 
 def llm_synchronize(m):

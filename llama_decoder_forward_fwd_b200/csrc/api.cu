@@ -153,6 +153,7 @@ struct llm_model {
     CUtensorMap* d_tmaps = nullptr;
     const void** d_norms = nullptr;
     unsigned* ds_bar = nullptr;
+    unsigned* probe_cnt = nullptr;  // grid-barrier counter of the wait probe
     // per-launch CUDA-event timing (LLM_FLAG_KERNEL_TIMING)
     bool timing = false;
     bool capturing = false;
@@ -822,6 +823,7 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
     MALLOC_OR_BAIL(m->seq_len, (size_t)c.max_batch * 4);
     if (c.has_embed_and_head) MALLOC_OR_BAIL(m->d_logits, (size_t)c.max_batch * c.vocab * 4);
     MALLOC_OR_BAIL(m->d_err, 64);
+    MALLOC_OR_BAIL(m->probe_cnt, 16);
     if (c.flags & LLM_FLAG_DEBUG_TAPS) MALLOC_OR_BAIL(m->taps, (size_t)c.n_layers * Mx * D * 4);
 
     if (cudaMemsetAsync(m->am_counter, 0, 64, m->stream) != cudaSuccess ||
@@ -1109,6 +1111,14 @@ int llm_kernel_times(llm_model* m, int n, double* total_ms, int64_t* launches, i
             m->kt_ms[i] = 0.0;
             m->kt_n[i] = 0;
         }
+    return LLM_OK;
+}
+
+int llm_debug_wait_probe(llm_model* m, int which, double limit_ms) {
+    if (!m) return fail(LLM_ERR_NULL_PTR, "model is NULL");
+    if ((which != 0 && which != 1) || !(limit_ms > 0.0) || limit_ms > 10000.0)
+        return fail(LLM_ERR_BAD_ARG, "which must be 0 or 1 and limit_ms in (0, 10000]");
+    CK(launch_wait_probe(which, (uint64_t)(limit_ms * 1e6), m->d_err, m->probe_cnt, m->stream));
     return LLM_OK;
 }
 

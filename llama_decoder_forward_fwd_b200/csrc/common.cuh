@@ -25,6 +25,7 @@ enum : uint32_t {
     DERR_GRID_BARRIER_WAIT = 0x401,
     DERR_MK_PRODUCER_WAIT = 0x402,
     DERR_MK_CONSUMER_WAIT = 0x403,
+    DERR_PROBE_WAIT = 0x501,  // the wait probe (a wait that cannot complete)
 };
 
 // 4 seconds: far longer than any legitimate wait for one pipeline stage.
@@ -77,15 +78,16 @@ DEVI bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 // Bounded wait for the phase with the given parity to complete. Returns false
-// (after recording `code` in *err) if it did not complete within kWaitLimitNs.
-DEVI bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err, uint32_t code) {
+// (after recording `code` in *err) if it did not complete within limit_ns
+// (kWaitLimitNs unless a caller asks for another bound).
+DEVI bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err, uint32_t code, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             if (err) atomicCAS(err, 0u, code);
             return false;
         }
@@ -124,7 +126,8 @@ DEVI unsigned ld_acquire_gpu(const unsigned* p) {
 // arrival, acquire polling, CTA barrier). The wait is bounded: on timeout it records
 // `code` in *err and returns false; it also returns false as soon as *err
 // holds another CTA's error, so all CTAs leave promptly.
-DEVI bool grid_barrier(unsigned* count, unsigned index, int nthreads, uint32_t* err, uint32_t code) {
+DEVI bool grid_barrier(unsigned* count, unsigned index, int nthreads, uint32_t* err, uint32_t code,
+                       uint64_t limit_ns = kWaitLimitNs) {
     __shared__ int gb_ok;
     named_bar_sync(1, nthreads);
     if (threadIdx.x == 0) {
@@ -140,7 +143,7 @@ DEVI bool grid_barrier(unsigned* count, unsigned index, int nthreads, uint32_t* 
                     ok = 0;
                     break;
                 }
-                if (globaltimer() - t0 > kWaitLimitNs) {
+                if (globaltimer() - t0 > limit_ns) {
                     atomicCAS(err, 0u, code);
                     ok = 0;
                     break;

@@ -266,6 +266,12 @@ cudaError_t launch_finish_hidden(const float* h, float* h_out, long long n, int3
 cudaError_t launch_rope_tables(float* cosv, float* sinv, int n_pos, int half, double theta, int head_dim,
                                cudaStream_t s);
 
+// A wait that cannot complete, bounded by limit_ns, on the library's own wait
+// code: which = 0 an mbarrier expecting bytes that never arrive (one CTA),
+// which = 1 a grid barrier of a cooperative launch of two CTAs whose target
+// counts three arrivals. Either records its code in *err and returns.
+cudaError_t launch_wait_probe(int which, uint64_t limit_ns, uint32_t* err, unsigned* counter, cudaStream_t s);
+
 // Record msg as the calling thread's last error (llm_last_error) and return code.
 int set_error(int code, const char* msg);
 

@@ -110,4 +110,47 @@ cudaError_t launch_rope_tables(float* cosv, float* sinv, int n_pos, int half, do
     return cudaGetLastError();
 }
 
+// ---- wait probe: the bounded-wait path run on purpose ------------------
+// An mbarrier armed for 16 bytes that no copy delivers: the bounded wait gives
+// up after limit_ns, records DERR_PROBE_WAIT and returns. Nothing is left in
+// flight (no copy was issued), so the CTA retires normally.
+__global__ void wait_probe_mbar_kernel(uint64_t limit_ns, uint32_t* err) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(&bar, 16);
+        mbar_wait(&bar, 0, err, DERR_PROBE_WAIT, limit_ns);
+    }
+}
+// A grid barrier that is never reached: each CTA arrives once (the counter
+// starts at zero), but barrier index 1 waits for 2 * gridDim.x arrivals. The
+// first CTA to give up after limit_ns records DERR_PROBE_WAIT; the other sees the
+// error word and leaves too.
+__global__ void wait_probe_grid_kernel(uint64_t limit_ns, uint32_t* err, unsigned* counter) {
+    grid_barrier(counter, 1, blockDim.x, err, DERR_PROBE_WAIT, limit_ns);
+}
+
+cudaError_t launch_wait_probe(int which, uint64_t limit_ns, uint32_t* err, unsigned* counter, cudaStream_t s) {
+    if (which == 0) {
+        wait_probe_mbar_kernel<<<1, 32, 0, s>>>(limit_ns, err);
+        return cudaGetLastError();
+    }
+    if (which != 1 || !counter) return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(counter, 0, 4, s);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(32);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;  // both CTAs resident: the wait is the only thing that stops them
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, wait_probe_grid_kernel, limit_ns, err, counter);
+    if (e != cudaSuccess) return e;
+    return cudaMemsetAsync(counter, 0, 4, s);
+}
+
 }  // namespace lfw

@@ -58,6 +58,7 @@ def test_null_arguments_are_rejected_on_the_host(lib):
     assert h.value is None
     assert lib.llm_model_init(None, None, None, None) == L.LLM_ERR_NULL_PTR
     assert b"NULL" in lib.llm_last_error()
+    assert lib.llm_debug_wait_probe(None, 0, ctypes.c_double(1.0)) == L.LLM_ERR_NULL_PTR
     assert lib.llm_prefill(None, None, 1, 1, None, None) == L.LLM_ERR_NULL_PTR
     assert lib.llm_decode_step(None, 1, None, None, None) == L.LLM_ERR_NULL_PTR
     assert lib.llm_kv_cache_reset(None) == L.LLM_ERR_NULL_PTR
