@@ -298,13 +298,13 @@ int llm_op_attention_decode(const void* q, const void* kcache, const void* vcach
  * 0..pos0[b] of q[b][h] . K[b][h/G][j] / sqrt(128), times V[b][h/G][j].
  *   q, out: [B][H*128] bf16; kcache, vcache: [B][Hk][S_max][128] bf16 holding
  *   positions 0..pos0[b] (the new token's key and value included); pos0: [B]
- *   int32 (0 <= pos0[b] < S_max). G = H / Hk must be at most 8. Device
- *   pointers, 16-byte aligned, owned by the caller; no workspace: a thread-block
- *   cluster per (sequence, KV head) streams 32-key K/V tiles by TMA and merges
- *   its CTAs' partial results in distributed shared memory. The probabilities
- *   enter the P V product rounded to bf16 (fp32 accumulation).
- *   Errors: LLM_ERR_NULL_PTR, LLM_ERR_BAD_ARG (shape, alignment),
- *   LLM_ERR_UNSUPPORTED (G > 8), LLM_ERR_CUDA.
+ *   int32 (0 <= pos0[b] < S_max); H a multiple of Hk. Device pointers,
+ *   16-byte aligned, owned by the caller; no workspace: a thread-block cluster
+ *   per (sequence, KV head, up to 8 of its query heads) streams 32-key K/V
+ *   tiles by TMA and merges its CTAs' partial results in distributed shared
+ *   memory. The probabilities enter the P V product rounded to bf16 (fp32
+ *   accumulation).
+ *   Errors: LLM_ERR_NULL_PTR, LLM_ERR_BAD_ARG (shape, alignment), LLM_ERR_CUDA.
  */
 int llm_op_attention_decode_cluster(const void* q, const void* kcache, const void* vcache,
                                     const int32_t* pos0, void* out, int B, int H, int Hk,

@@ -865,8 +865,10 @@ int llm_model_init(const llm_config* cfg, const llm_weights* w, void* stream, ll
         if (ok) ok = make_tmap(&m->tm_hw, m->hw, D, Mx, 64, 128) && make_tmap(&m->tm_o, m->o, H * d, Mx, 64, 128) &&
                      make_tmap(&m->tm_g, m->g, F, Mx, 64, 128);
         if (!ok) return bail(fail(LLM_ERR_CUDA, "cuTensorMapEncodeTiled failed"));
-        m->gemm_ok = D % GEMM_BN == 0 && (H * d) % GEMM_BN == 0 && (Hk * d) % GEMM_BN == 0 &&
-                     F % (GEMM_BN / 2) == 0 && D % GEMM_BK == 0 && F % GEMM_BK == 0 && (H * d) % GEMM_BK == 0;
+        // the QKV output in whole 256-column tiles, each half from one of wq, wk, wv
+        m->gemm_ok = D % GEMM_BN == 0 && (H * d) % (GEMM_BN / 2) == 0 && (Hk * d) % (GEMM_BN / 2) == 0 &&
+                     ((H + 2 * Hk) * d) % GEMM_BN == 0 && F % (GEMM_BN / 2) == 0 && D % GEMM_BK == 0 &&
+                     F % GEMM_BK == 0 && (H * d) % GEMM_BK == 0;
         if (d == 128) {
             const uint64_t rows = (uint64_t)c.n_layers * c.max_batch * Hk * c.max_seq_len;
             if (!make_tmap(&m->tm_kc, m->kc, d, rows, 64, 64) || !make_tmap(&m->tm_vc, m->vc, d, rows, 64, 64) ||
@@ -1298,7 +1300,7 @@ int llm_op_attention_decode_cluster(const void* q, const void* kcache, const voi
     int rc = lfw::attn_op_check(q, kcache, vcache, pos0, out, B, 1, H, Hk, 128, S_max, LLM_BF16);
     if (rc) return rc;
     const int cs = attn_cluster_size(B, H, Hk, 128, num_sms_current());
-    if (cs < 1) return fail(LLM_ERR_UNSUPPORTED, "cluster attention needs at most 8 query heads per KV head");
+    if (cs < 1) return fail(LLM_ERR_UNSUPPORTED, "cluster attention does not support this shape");
     CUtensorMap tk, tv;
     const uint64_t rows = (uint64_t)B * Hk * S_max;
     if (!make_tmap(&tk, kcache, 128, rows, 64, 32) || !make_tmap(&tv, vcache, 128, rows, 64, 32))

@@ -6,8 +6,10 @@
 // keys 0 .. p (p the new token's position) of KV head h / G, scores q.k /
 // sqrt(d), softmax, weighted sum of values.
 //
-// A group's keys are cut into 32-key units (the K and V tiles of 32 positions,
-// 16 KB) and split evenly over the cs CTAs of its cluster. In each CTA a producer
+// A group is a sequence's KV head with up to 8 of its query heads (a KV head
+// with more, as in multi-query attention, makes several groups, each reading
+// the head's keys and values). Its keys are cut into 32-key units (the K and V
+// tiles of 32 positions, 16 KB) and split evenly over the cs CTAs of its cluster. In each CTA a producer
 // warp streams the CTA's units by TMA into a ring of shared-memory stages (one
 // copy of each tile, shared by all the group's query heads), and the eight
 // consumer warps take the units in turn, computing S = Q K^T, an online softmax
@@ -85,7 +87,12 @@ __global__ void __launch_bounds__(AC_THREADS, 1)
     uint64_t* empty = full + AC_STAGES;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = a.cs > 1 ? cluster_ctarank() : 0u;
-    const int gr = blockIdx.y, b = gr / a.Hk, kvh = gr % a.Hk, R = a.H / a.Hk;
+    // group: (sequence, KV head, chunk of at most 8 of its query heads)
+    const int G = a.H / a.Hk, chunks = (G + AC_RMAX - 1) / AC_RMAX;
+    const int gr = blockIdx.y / chunks, chunk = blockIdx.y % chunks;
+    const int b = gr / a.Hk, kvh = gr % a.Hk;
+    const int R = G - chunk * AC_RMAX < AC_RMAX ? G - chunk * AC_RMAX : AC_RMAX;
+    const int head0 = kvh * G + chunk * AC_RMAX;  // first query head of the group
     int p0 = a.pos0[b];
     p0 = p0 < 0 ? 0 : (p0 >= a.S_max ? a.S_max - 1 : p0);
     const int U = (p0 + AK) / AK;  // units covering keys 0 .. p0
@@ -127,7 +134,7 @@ __global__ void __launch_bounds__(AC_THREADS, 1)
         __syncwarp();
     } else {
         // consumers: the group's query rows, then units i = warp, warp + 8, ...
-        attn_q_tile(scratch, a.q + (size_t)b * a.H * 128 + (size_t)kvh * R * 128, 128, R, threadIdx.x);
+        attn_q_tile(scratch, a.q + (size_t)b * a.H * 128 + (size_t)head0 * 128, 128, R, threadIdx.x);
         named_bar_sync(1, AC_CONSUMERS);
         float* wst = reinterpret_cast<float*>(scratch + 4096);
         AttnAcc acc;
@@ -147,7 +154,7 @@ __global__ void __launch_bounds__(AC_THREADS, 1)
             float M, L, O[4];
             attn_merge_warps<AC_CONSUMERS / 32>(wst, R, r, d4, M, L, O);
             if (a.cs == 1) {
-                attn_out4(a, b * a.H * 128 + (kvh * R + r) * 128 + d4, O, L);
+                attn_out4(a, b * a.H * 128 + (head0 + r) * 128 + d4, O, L);
             } else {
                 float* pr = piece + r * AW_REC;
                 *reinterpret_cast<float4*>(pr + 4 + d4) = make_float4(O[0], O[1], O[2], O[3]);
@@ -181,14 +188,16 @@ __global__ void __launch_bounds__(AC_THREADS, 1)
             if (q >= a.cs) break;
             lse_merge(M, L, O, mp[q], lp[q], op[q]);
         }
-        attn_out4(a, b * a.H * 128 + (kvh * R + r) * 128 + d4, O, L);
+        attn_out4(a, b * a.H * 128 + (head0 + r) * 128 + d4, O, L);
     }
     cluster_sync_all();  // every piece stays in place until the first CTA has read it
 }
 
+int attn_cluster_groups(int B, int H, int Hk) { return B * Hk * ((H / Hk + AC_RMAX - 1) / AC_RMAX); }
+
 int attn_cluster_size(int B, int H, int Hk, int d, int num_sms) {
-    if (d != 128 || Hk < 1 || H % Hk != 0 || H / Hk > AC_RMAX || B < 1) return 0;
-    const int groups = B * Hk;
+    if (d != 128 || Hk < 1 || H % Hk != 0 || B < 1) return 0;
+    const int groups = attn_cluster_groups(B, H, Hk);
     int cs = 1;
     while (cs < 8 && groups * cs < num_sms) cs *= 2;
     return cs;
@@ -196,8 +205,7 @@ int attn_cluster_size(int B, int H, int Hk, int d, int num_sms) {
 
 cudaError_t launch_attn_cluster(const AttnClusterArgs& a, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                 cudaStream_t s) {
-    if (a.cs < 1 || a.cs > 8 || a.H % a.Hk != 0 || a.H / a.Hk > AC_RMAX || !tmK || !tmV)
-        return cudaErrorInvalidValue;
+    if (a.cs < 1 || a.cs > 8 || a.Hk < 1 || a.H % a.Hk != 0 || !tmK || !tmV) return cudaErrorInvalidValue;
     static bool attr = false;
     if (!attr) {
         const cudaError_t e = cudaFuncSetAttribute(attn_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -206,7 +214,7 @@ cudaError_t launch_attn_cluster(const AttnClusterArgs& a, const CUtensorMap* tmK
         attr = true;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.cs, a.B * a.Hk);
+    cfg.gridDim = dim3(a.cs, attn_cluster_groups(a.B, a.H, a.Hk));
     cfg.blockDim = dim3(AC_THREADS);
     cfg.dynamicSmemBytes = AC_SMEM;
     cfg.stream = s;

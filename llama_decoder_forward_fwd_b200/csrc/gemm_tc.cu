@@ -98,14 +98,18 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                     b1 = &tmB1;
                     r0 = r1 = nb * (GEMM_BN / 2);
                 } else {
-                    int c = nb * GEMM_BN, s = 0;
-                    while (s < 2 && c >= p.seg_cols[s]) {
-                        c -= p.seg_cols[s];
-                        ++s;
-                    }
-                    b0 = b1 = (s == 0) ? &tmB0 : (s == 1) ? &tmB1 : &tmB2;
-                    r0 = c;
-                    r1 = c + GEMM_BN / 2;
+                    // each 128-row half of the tile from the segment (wq, wk, wv) holding it
+                    auto seg_of = [&](int c, int& row) -> const CUtensorMap* {
+                        int s = 0;
+                        while (s < 2 && c >= p.seg_cols[s]) {
+                            c -= p.seg_cols[s];
+                            ++s;
+                        }
+                        row = c;
+                        return (s == 0) ? &tmB0 : (s == 1) ? &tmB1 : &tmB2;
+                    };
+                    b0 = seg_of(nb * GEMM_BN, r0);
+                    b1 = seg_of(nb * GEMM_BN + GEMM_BN / 2, r1);
                 }
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, err, DERR_GEMM_PRODUCER_WAIT)) {

@@ -175,8 +175,8 @@ AttnDecodePlan attn_decode_plan(int B, int T, int H, int Hk, int d, int max_keys
 cudaError_t launch_attn_decode(const AttnDecodeArgs& a, bool bf16, cudaStream_t s, bool pdl);
 
 // Decode attention of one new token per sequence on the tensor cores, one
-// thread-block cluster per (sequence, KV head) group (attn_cluster.cu): bf16,
-// head_dim 128, at most 8 query heads per KV head. Needs no global scratch.
+// thread-block cluster per group of up to 8 query heads of one (sequence, KV
+// head) (attn_cluster.cu): bf16, head_dim 128. Needs no global scratch.
 struct AttnClusterArgs {
     const __nv_bfloat16* q = nullptr;  // [B][H*128]
     __nv_bfloat16* out = nullptr;      // [B][H*128]
@@ -189,7 +189,8 @@ struct AttnClusterArgs {
     float scale_log2 = 0.f;
     uint32_t* err = nullptr;
 };
-// CTAs per group for B sequences of Hk KV heads on num_sms SMs (0: shape not supported).
+// Groups of the launch, and CTAs per group on num_sms SMs (0: shape not supported).
+int attn_cluster_groups(int B, int H, int Hk);
 int attn_cluster_size(int B, int H, int Hk, int d, int num_sms);
 // tmK, tmV: the K and V caches as [rows][128] bf16 with 32-row, 64-column boxes.
 cudaError_t launch_attn_cluster(const AttnClusterArgs& a, const CUtensorMap* tmK, const CUtensorMap* tmV,

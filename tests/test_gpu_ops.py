@@ -126,6 +126,9 @@ def test_split_kv_attention_matches_oracle(lib, dtype, d, tol, B, T, H, Hk, pos0
     (8, 32, 32, 1152, [1024 + i for i in range(8)]),   # multi-head attention: one query head per KV head
     (2, 16, 2, 512, [100, 3]),         # 8 query heads per KV head
     (2, 12, 4, 300, [299, 150]),       # 3 query heads per KV head, a cache of 300 positions
+    (1, 32, 1, 1024, [700]),           # multi-query: 4 groups of 8 query heads read the one KV head
+    (2, 24, 1, 512, [100, 3]),         # 24 query heads per KV head: 3 groups of 8
+    (1, 20, 2, 256, [255]),            # 10 per KV head: groups of 8 and 2
 ])
 def test_cluster_decode_attention_matches_oracle(lib, B, H, Hk, S, pos0):
     """The tensor-core decode attention (one cluster per KV-head group, pieces merged
@@ -141,16 +144,6 @@ def test_cluster_decode_attention_matches_oracle(lib, B, H, Hk, S, pos0):
     torch.cuda.synchronize()
     err = np.abs(O.f64(out.cpu()) - ref)
     assert err.max() <= 8e-3 * float(vc.abs().max()), err.max()
-
-
-def test_cluster_decode_attention_rejects_large_groups(lib):
-    import llama_decoder_forward_fwd_b200 as L
-    q = torch.zeros(1, 1, 32 * 128, dtype=torch.bfloat16, device=DEV)
-    kc = torch.zeros(1, 1, 64, 128, dtype=torch.bfloat16, device=DEV)
-    p = torch.zeros(1, dtype=torch.int32, device=DEV)
-    with pytest.raises(L.LlmError) as e:
-        L.llm_op_attention_decode_cluster(q.view(1, 1, 32, 128), kc, kc, p, q)
-    assert e.value.code == L.LLM_ERR_UNSUPPORTED
 
 
 def test_split_kv_attention_batch_16_long_caches_matches_oracle(lib):
