@@ -62,10 +62,6 @@ DEVI void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
 DEVI void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-// Arrive `count` times at once (one thread standing for several consumers).
-DEVI void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
 DEVI bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
