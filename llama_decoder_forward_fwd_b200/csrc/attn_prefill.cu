@@ -1,4 +1,5 @@
-// Causal grouped-query attention for a block of prompt tokens (prefill).
+// Causal grouped-query attention for a block of prompt tokens (prefill), on the
+// 5th-generation tensor cores.
 //
 // What it computes ("Resumen ...", "Implementación de la atención" and
 // "Atención multi-head"; llama3.np, "GQA" and "Scaled Dot-Product Attention"):
@@ -9,11 +10,23 @@
 // Layout of the work. A CTA owns 128 "rows" of one (sequence, KV head): row r is
 // (token t = r / G, query head kvh*G + r % G), so the G query heads that share a
 // KV head sit in one CTA and every K/V tile is loaded once for all of them.
-// K and V tiles of 64 keys x 128 dims come from the KV cache by TMA (two
-// 64-dim halves with the 128-byte swizzle) into a 2-stage ring. Each of the 8
-// warps runs mma.sync m16n8k16 on its 16 rows: S = Q K^T (ldmatrix from the
-// swizzled tiles), an online softmax in registers (running max and sum in the
-// log2 domain), and O += P V with P reused from the S registers.
+// Keys go in tiles of 128, d = 128. Six warps:
+//   warp 0     TMA producer: K and V tiles (two 64-dim halves, 128-byte swizzle)
+//              from the KV cache into 2-stage rings, K and V on their own barriers;
+//   warp 1     allocates 512 TMEM columns and issues tcgen05.mma from one thread:
+//              S = Q K^T (M = 128 rows, N = 128 keys, K = d) into one of two S
+//              accumulators, and O += P V (N = d, K = keys; V read MN-major, as it
+//              lies in the cache) into the O accumulator;
+//   warps 2-5  softmax, one thread per row (its TMEM lane): tcgen05.ld of the row
+//              of S, scale and causal mask, running maximum in the log2 domain,
+//              P = 2^(s - m) stored to shared memory in bf16 as the A operand of
+//              the PV product, running sum; at the end tcgen05.ld of O / sum.
+// The MMA thread issues S for tile j+2 as soon as P of tile j is written, so the
+// tensor cores compute the next scores while the softmax warps work.
+// O is rescaled (tcgen05.ld, scale, tcgen05.st) only when a row's maximum grows
+// by more than 2^8 over the maximum its P values were taken against (the
+// conditional rescaling of FlashAttention-4): P stays below 256, exact in the
+// final normalisation, which divides by a sum taken against the same maximum.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -21,66 +34,75 @@
 
 namespace lfw {
 
-constexpr int FA_THREADS = 256;
+constexpr int FA_THREADS = 192;
 constexpr int FA_ROWS = 128;
-constexpr int FA_KT = 64;
+constexpr int FA_KT = 128;                      // keys per tile
 constexpr int FA_D = 128;
-constexpr int FA_Q_BYTES = FA_ROWS * FA_D * 2;   // 32 KB
-constexpr int FA_KV_BYTES = FA_KT * FA_D * 2;    // 16 KB per K or V tile
-constexpr int FA_SMEM = 1024 + FA_Q_BYTES + 4 * FA_KV_BYTES + 64;
-
-DEVI uint32_t kv_addr(uint32_t base, int key, int chunk) {
-    // chunk: 16-byte column chunk 0..15 of the 128-dim row; halves are 8 KB apart.
-    return base + (chunk >> 3) * (FA_KT * 128) + key * 128 + (((chunk & 7) ^ (key & 7)) << 4);
-}
+constexpr int FA_HALF = 128 * 128;              // [128 rows][64 bf16]: 16 KB
+constexpr int FA_TILE = 2 * FA_HALF;            // a K, V, Q or P tile: 32 KB
+constexpr int FA_SMEM = 1024 + 6 * FA_TILE + 256;
+constexpr uint32_t FA_TMEM_COLS = 512;          // S (2 x 128 columns), O (128)
+constexpr uint32_t FA_TMEM_O = 256;
+constexpr float FA_RESCALE_LOG2 = 8.f;
 
 __global__ void __launch_bounds__(FA_THREADS, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const AttnPrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* Ks = smem;                       // 2 stages x 16 KB
-    uint8_t* Vs = smem + 2 * FA_KV_BYTES;     // 2 stages x 16 KB
-    uint8_t* Qs = smem + 4 * FA_KV_BYTES;     // 32 KB
-    uint64_t* barK = reinterpret_cast<uint64_t*>(Qs + FA_Q_BYTES);
-    uint64_t* barV = barK + 2;
+    // V stages sit below Q and P, so every operand read stays inside the allocation.
+    uint8_t* Ks = smem;                  // 2 stages
+    uint8_t* Vs = smem + 2 * FA_TILE;    // 2 stages
+    uint8_t* Qs = smem + 4 * FA_TILE;
+    uint8_t* Ps = smem + 5 * FA_TILE;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 6 * FA_TILE);
+    uint64_t* k_full = bars;
+    uint64_t* k_empty = bars + 2;
+    uint64_t* v_full = bars + 4;
+    uint64_t* v_empty = bars + 6;
+    uint64_t* s_full = bars + 8;
+    uint64_t* p_full = bars + 10;
+    uint64_t* pv_done = bars + 11;
+    uint64_t* mma_done = bars + 12;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, t4 = lane & 3;
     const int G = a.H / a.Hk;
     const int rb = gridDim.x - 1 - blockIdx.x;  // longest rows first
     const int b = blockIdx.y / a.Hk, kvh = blockIdx.y % a.Hk;
-    const int HD = a.H * FA_D;
+    uint32_t* err = a.err;
+
+    if (warp == 0 && lane == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&k_full[i], 1);
+            mbar_init(&k_empty[i], 1);
+            mbar_init(&v_full[i], 1);
+            mbar_init(&v_empty[i], 1);
+            mbar_init(&s_full[i], 1);
+        }
+        mbar_init(p_full, 128);
+        mbar_init(pv_done, 1);
+        mbar_init(mma_done, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    if (warp == 1) {
+        tc_alloc(tmem_slot, FA_TMEM_COLS);
+        tc_relinquish();
+    }
 
     pdl_trigger();
     pdl_wait();
     const int p0 = a.pos0[b];
-
     const int row0 = rb * FA_ROWS;
     const int t_last = min(a.T - 1, (row0 + FA_ROWS - 1) / G);
-    const int p_max = min(p0 + t_last, a.S_max - 1);  // never read past this head's cache rows
+    const int p_max = min(p0 + t_last, a.S_max - 1);  // the last key any row of this CTA sees
     const int nkt = p_max / FA_KT + 1;
     const long long kv_row0 = a.row_base + (long long)(b * a.Hk + kvh) * a.S_max;
 
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&barK[i], 1);
-            mbar_init(&barV[i], 1);
-        }
-        fence_mbar_init();
-        tma_prefetch_desc(&tmK);
-        tma_prefetch_desc(&tmV);
-        for (int kt = 0; kt < 2 && kt < nkt; ++kt) {
-            mbar_arrive_expect_tx(&barK[kt], FA_KV_BYTES);
-            tma_load_2d(Ks + kt * FA_KV_BYTES, &tmK, &barK[kt], 0, (int)(kv_row0 + kt * FA_KT));
-            tma_load_2d(Ks + kt * FA_KV_BYTES + FA_KV_BYTES / 2, &tmK, &barK[kt], 64, (int)(kv_row0 + kt * FA_KT));
-            mbar_arrive_expect_tx(&barV[kt], FA_KV_BYTES);
-            tma_load_2d(Vs + kt * FA_KV_BYTES, &tmV, &barV[kt], 0, (int)(kv_row0 + kt * FA_KT));
-            tma_load_2d(Vs + kt * FA_KV_BYTES + FA_KV_BYTES / 2, &tmV, &barV[kt], 64, (int)(kv_row0 + kt * FA_KT));
-        }
-    }
-
-    // Stage this CTA's 128 query rows in shared memory (16-byte chunks XOR-swizzled by row).
+    // Stage this CTA's 128 query rows as the A operand of S = Q K^T: two 64-dim
+    // halves of [128 rows][128 bytes], 16-byte chunks XOR-swizzled by row.
     for (int idx = threadIdx.x; idx < FA_ROWS * 16; idx += FA_THREADS) {
         const int r = idx >> 4, c = idx & 15;
         const int rg = row0 + r;
@@ -88,153 +110,209 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         uint4 v = make_uint4(0, 0, 0, 0);
         if (t < a.T)
             v = *reinterpret_cast<const uint4*>(a.q + ((long long)(b * a.T + t) * a.H + h) * FA_D + c * 8);
-        *reinterpret_cast<uint4*>(Qs + r * 256 + ((c ^ (r & 7)) << 4)) = v;
+        *reinterpret_cast<uint4*>(Qs + (c >> 3) * FA_HALF + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
     }
+    fence_proxy_async();  // the tensor cores read Q through the async proxy
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
 
-    uint32_t qf[8][4];
-    {
-        const uint32_t qbase = smem_u32(Qs);
-        const int j = lane >> 3, i = lane & 7;
-        const int r = warp * 16 + (j & 1) * 8 + i;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const int c = 2 * kk + (j >> 1);
-            ldsm_x4(qf[kk], qbase + r * 256 + ((c ^ (r & 7)) << 4));
-        }
-    }
-
-    // Positions of this lane's two rows (g and g+8 of the warp's 16); -1 if no token.
-    int prow[2];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        const int rg = row0 + warp * 16 + g + 8 * hh;
-        const int t = rg / G;
-        prow[hh] = t < a.T ? p0 + t : -1;
-    }
-    const int wr_first = row0 + warp * 16, wr_last = row0 + warp * 16 + 15;
-    const int w_plo = (wr_first / G < a.T) ? p0 + wr_first / G : INT_MAX;
-    const int w_phi = (wr_first / G < a.T) ? p0 + min(a.T - 1, wr_last / G) : -1;
-
-    float o[16][4];
-#pragma unroll
-    for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-    float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
-    const float sl2 = a.scale_log2;
-    bool ok = true;
-
-    for (int kt = 0; kt < nkt; ++kt) {
-        const int st = kt & 1;
-        const uint32_t ph = (kt >> 1) & 1;
-        const bool active = ok && (kt * FA_KT <= w_phi);
-        if (ok && !mbar_wait(&barK[st], ph, a.err, DERR_ATTN_TMA_WAIT)) ok = false;
-        if (active && ok) {
-            const uint32_t kb = smem_u32(Ks + st * FA_KV_BYTES);
-            float s[8][4];
-#pragma unroll
-            for (int n = 0; n < 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
-            {
-                const int j = lane >> 3, i = lane & 7;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-                    for (int np = 0; np < 4; ++np) {
-                        uint32_t r[4];
-                        const int key = (2 * np + (j >> 1)) * 8 + i;
-                        ldsm_x4(r, kv_addr(kb, key, 2 * kk + (j & 1)));
-                        mma_bf16_16816(s[2 * np], qf[kk], r[0], r[1]);
-                        mma_bf16_16816(s[2 * np + 1], qf[kk], r[2], r[3]);
-                    }
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};  // last tile loaded into each stage
+            bool ok = true;
+            for (int j = 0; j < nkt && ok; ++j) {
+                const int st = j & 1;
+                const uint32_t ph = (j >> 1) & 1;
+                const int y = (int)(kv_row0 + (long long)j * FA_KT);
+                if (!mbar_wait(&k_empty[st], ph ^ 1u, err, DERR_ATTN_TMA_WAIT)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&k_full[st], FA_TILE);
+                for (int h = 0; h < 2; ++h)
+                    for (int kb = 0; kb < 2; ++kb)
+                        tma_load_2d(Ks + st * FA_TILE + h * FA_HALF + kb * (FA_HALF / 2), &tmK, &k_full[st], h * 64,
+                                    y + kb * 64);
+                last_k[st] = j;
+                if (!mbar_wait(&v_empty[st], ph ^ 1u, err, DERR_ATTN_TMA_WAIT)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&v_full[st], FA_TILE);
+                for (int h = 0; h < 2; ++h)
+                    for (int kb = 0; kb < 2; ++kb)
+                        tma_load_2d(Vs + st * FA_TILE + h * FA_HALF + kb * (FA_HALF / 2), &tmV, &v_full[st], h * 64,
+                                    y + kb * 64);
+                last_v[st] = j;
+            }
+            if (!ok) {
+                // let copies already issued land before the CTA can exit
+                for (int st = 0; st < 2; ++st) {
+                    if (last_k[st] >= 0) mbar_wait(&k_full[st], (last_k[st] >> 1) & 1, nullptr, 0);
+                    if (last_v[st] >= 0) mbar_wait(&v_full[st], (last_v[st] >> 1) & 1, nullptr, 0);
                 }
             }
-            const bool need_mask = (kt * FA_KT + FA_KT - 1) > w_plo;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float mx = -INFINITY;
-#pragma unroll
-                for (int n = 0; n < 8; ++n)
-#pragma unroll
-                    for (int e2 = 0; e2 < 2; ++e2) {
-                        float v = s[n][2 * hh + e2] * sl2;
-                        if (need_mask) {
-                            const int key = kt * FA_KT + n * 8 + 2 * t4 + e2;
-                            if (key > prow[hh]) v = -INFINITY;
-                        }
-                        s[n][2 * hh + e2] = v;
-                        mx = fmaxf(mx, v);
-                    }
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                const float mnew = fmaxf(mrow[hh], mx);
-                const float muse = (mnew == -INFINITY) ? 0.f : mnew;
-                const float alpha = exp2f(mrow[hh] - muse);
-                mrow[hh] = mnew;
-                float sum = 0.f;
-#pragma unroll
-                for (int n = 0; n < 8; ++n)
-#pragma unroll
-                    for (int e2 = 0; e2 < 2; ++e2) {
-                        const float pv = exp2f(s[n][2 * hh + e2] - muse);
-                        s[n][2 * hh + e2] = pv;
-                        sum += pv;
-                    }
-                lrow[hh] = lrow[hh] * alpha + sum;
-#pragma unroll
-                for (int n = 0; n < 16; ++n) {
-                    o[n][2 * hh] *= alpha;
-                    o[n][2 * hh + 1] *= alpha;
-                }
-            }
-            if (!mbar_wait(&barV[st], ph, a.err, DERR_ATTN_TMA_WAIT)) ok = false;
-            if (ok) {
-                const uint32_t vb = smem_u32(Vs + st * FA_KV_BYTES);
-                const int j = lane >> 3, i = lane & 7;
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    uint32_t pf[4];
-                    pf[0] = pack_bf16x2(s[2 * ks][0], s[2 * ks][1]);
-                    pf[1] = pack_bf16x2(s[2 * ks][2], s[2 * ks][3]);
-                    pf[2] = pack_bf16x2(s[2 * ks + 1][0], s[2 * ks + 1][1]);
-                    pf[3] = pack_bf16x2(s[2 * ks + 1][2], s[2 * ks + 1][3]);
-                    const int key = ks * 16 + (j & 1) * 8 + i;
-#pragma unroll
-                    for (int dp = 0; dp < 8; ++dp) {
-                        uint32_t r[4];
-                        ldsm_x4_t(r, kv_addr(vb, key, 2 * dp + (j >> 1)));
-                        mma_bf16_16816(o[2 * dp], pf, r[0], r[1]);
-                        mma_bf16_16816(o[2 * dp + 1], pf, r[2], r[3]);
-                    }
-                }
-            }
-        } else if (ok) {
-            if (!mbar_wait(&barV[st], ph, a.err, DERR_ATTN_TMA_WAIT)) ok = false;
         }
-        __syncthreads();
-        if (threadIdx.x == 0 && kt + 2 < nkt) {
-            const int nt = kt + 2;
-            mbar_arrive_expect_tx(&barK[st], FA_KV_BYTES);
-            tma_load_2d(Ks + st * FA_KV_BYTES, &tmK, &barK[st], 0, (int)(kv_row0 + nt * FA_KT));
-            tma_load_2d(Ks + st * FA_KV_BYTES + FA_KV_BYTES / 2, &tmK, &barK[st], 64, (int)(kv_row0 + nt * FA_KT));
-            mbar_arrive_expect_tx(&barV[st], FA_KV_BYTES);
-            tma_load_2d(Vs + st * FA_KV_BYTES, &tmV, &barV[st], 0, (int)(kv_row0 + nt * FA_KT));
-            tma_load_2d(Vs + st * FA_KV_BYTES + FA_KV_BYTES / 2, &tmV, &barV[st], 64, (int)(kv_row0 + nt * FA_KT));
-        }
-    }
-
-    // Normalise and store this lane's two rows.
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16_f32(FA_ROWS, FA_KT);
+            constexpr uint32_t idO = idesc_bf16_f32_bmn(FA_ROWS, FA_D);
+            const uint32_t qa = smem_u32(Qs), pa = smem_u32(Ps);
+            auto issue_s = [&](int j) -> bool {
+                const int st = j & 1;
+                if (!mbar_wait(&k_full[st], (j >> 1) & 1, err, DERR_ATTN_MMA_WAIT)) return false;
+                tc_fence_after();
+                const uint32_t ka = smem_u32(Ks + st * FA_TILE);
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        float l = lrow[hh];
-        l += __shfl_xor_sync(0xffffffffu, l, 1);
-        l += __shfl_xor_sync(0xffffffffu, l, 2);
-        const int rg = row0 + warp * 16 + g + 8 * hh;
+                for (int kk = 0; kk < FA_D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * FA_HALF + (kk & 3) * 32;
+                    tc_mma_f16(tmem_base + st * FA_KT, smem_desc_sw128(qa + off), smem_desc_sw128(ka + off), idS,
+                               kk != 0);
+                }
+                tc_commit(&k_empty[st]);
+                tc_commit(&s_full[st]);
+                return true;
+            };
+            bool ok = issue_s(0);
+            if (ok && nkt > 1) ok = issue_s(1);
+            for (int j = 0; j < nkt && ok; ++j) {
+                const int st = j & 1;
+                if (!mbar_wait(p_full, j & 1, err, DERR_ATTN_MMA_WAIT)) break;
+                if (!mbar_wait(&v_full[st], (j >> 1) & 1, err, DERR_ATTN_MMA_WAIT)) break;
+                tc_fence_after();
+                const uint32_t va = smem_u32(Vs + st * FA_TILE);
+#pragma unroll
+                for (int kk = 0; kk < FA_KT / 16; ++kk) {
+                    // A = P: keys 16kk.. of the K-major P tile; B = V: the same 16 key rows,
+                    // all 128 dims (the second 64-dim half FA_HALF bytes on)
+                    tc_mma_f16(tmem_base + FA_TMEM_O, smem_desc_sw128(pa + (kk >> 2) * FA_HALF + (kk & 3) * 32),
+                               smem_desc_sw128_mn(va + kk * 2048, FA_HALF), idO, (j | kk) != 0);
+                }
+                tc_commit(&v_empty[st]);
+                tc_commit(pv_done);
+                if (j + 2 < nkt) ok = issue_s(j + 2);
+            }
+            tc_commit(mma_done);  // arrives once every MMA issued above has completed
+        }
+    } else {
+        // ---------------- softmax (warps 2..5), one thread per row ----------------
+        const int q4 = warp & 3;  // the TMEM lane quarter this warp may access
+        const int r = q4 * 32 + lane;
+        const int rg = row0 + r;
         const int t = rg / G, h = kvh * G + (rg - t * G);
-        if (t >= a.T || prow[hh] < 0) continue;
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        __nv_bfloat16* dst = a.out + (long long)(b * a.T + t) * HD + h * FA_D + 2 * t4;
+        const int prow = t < a.T ? p0 + t : -1;
+        const uint32_t lane_base = tmem_base + ((uint32_t)(q4 * 32) << 16);
+        const float sl2 = a.scale_log2;
+        float m_used = -INFINITY, l = 0.f;
+        bool ok = true;
+        uint8_t* prow_s = Ps + r * 128;
+        for (int j = 0; j < nkt; ++j) {
+            const int sb = j & 1;
+            if (ok && !mbar_wait(&s_full[sb], (j >> 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
+            tc_fence_after();
+            float s[FA_KT];
+            {
+                uint32_t u[4][32];
 #pragma unroll
-        for (int n = 0; n < 16; ++n)
-            *reinterpret_cast<uint32_t*>(dst + n * 8) = pack_bf16x2(o[n][2 * hh] * inv, o[n][2 * hh + 1] * inv);
+                for (int c = 0; c < 4; ++c) tc_ld_32x32b_x32(lane_base + sb * FA_KT + c * 32, u[c]);
+                tc_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(u[c][i]);
+            }
+            const int key0 = j * FA_KT;
+            float mx = -INFINITY;
+            if (key0 + FA_KT - 1 <= prow) {
+#pragma unroll
+                for (int i = 0; i < FA_KT; ++i) {
+                    s[i] *= sl2;
+                    mx = fmaxf(mx, s[i]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < FA_KT; ++i) {
+                    s[i] = key0 + i <= prow ? s[i] * sl2 : -INFINITY;
+                    mx = fmaxf(mx, s[i]);
+                }
+            }
+            const float m_new = fmaxf(m_used, mx);
+            const bool need = m_new > m_used + FA_RESCALE_LOG2;  // false while the row has seen no key
+            const float alpha = need ? exp2f(m_used - m_new) : 1.f;
+            if (j > 0) {
+                // PV of the previous tile has completed: O is stable and the P buffer free
+                if (ok && !mbar_wait(pv_done, (j - 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t u[32];
+                        tc_ld_32x32b_x32(lane_base + FA_TMEM_O + c * 32, u);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+                        tc_st_32x32b_x32(lane_base + FA_TMEM_O + c * 32, u);
+                    }
+                    tc_wait_st();
+                }
+            }
+            if (need) {
+                l *= alpha;
+                m_used = m_new;
+            }
+            const float muse = m_used == -INFINITY ? 0.f : m_used;
+            float sum = 0.f;
+#pragma unroll
+            for (int c = 0; c < FA_KT / 8; ++c) {
+                float p[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    p[e] = exp2f(s[c * 8 + e] - muse);
+                    sum += p[e];
+                }
+                const uint4 v = make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
+                                           pack_bf16x2(p[6], p[7]));
+                *reinterpret_cast<uint4*>(prow_s + (c >> 3) * FA_HALF + (((c & 7) ^ (r & 7)) << 4)) = v;
+            }
+            l += sum;
+            fence_proxy_async();  // P is read by the tensor cores through the async proxy
+            tc_fence_before();
+            mbar_arrive(p_full);
+        }
+        if (ok && !mbar_wait(pv_done, (nkt - 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
+        tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        __nv_bfloat16* dst = a.out + ((long long)(b * a.T + t) * a.H + h) * FA_D;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            uint32_t u[32];
+            tc_ld_32x32b_x32(lane_base + FA_TMEM_O + c * 32, u);
+            tc_wait_ld();
+            if (prow >= 0) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 8) {
+                    const uint4 v = make_uint4(pack_bf16x2(__uint_as_float(u[i]) * inv, __uint_as_float(u[i + 1]) * inv),
+                                               pack_bf16x2(__uint_as_float(u[i + 2]) * inv, __uint_as_float(u[i + 3]) * inv),
+                                               pack_bf16x2(__uint_as_float(u[i + 4]) * inv, __uint_as_float(u[i + 5]) * inv),
+                                               pack_bf16x2(__uint_as_float(u[i + 6]) * inv, __uint_as_float(u[i + 7]) * inv));
+                    *reinterpret_cast<uint4*>(dst + c * 32 + i) = v;
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        // every MMA has completed before the accumulators are freed
+        if (lane == 0) mbar_wait(mma_done, 0, err, DERR_ATTN_MMA_WAIT);
+        __syncwarp();
+        tc_fence_after();
+        tc_dealloc(tmem_base, FA_TMEM_COLS);
     }
 }
 

@@ -20,6 +20,8 @@ enum : uint32_t {
     DERR_GEMM_MMA_WAIT = 0x102,
     DERR_GEMM_EPI_WAIT = 0x103,
     DERR_ATTN_TMA_WAIT = 0x201,
+    DERR_ATTN_MMA_WAIT = 0x202,
+    DERR_ATTN_SOFTMAX_WAIT = 0x203,
     DERR_GEMV_PRODUCER_WAIT = 0x301,
     DERR_GEMV_CONSUMER_WAIT = 0x302,
     DERR_GRID_BARRIER_WAIT = 0x401,
@@ -209,6 +211,20 @@ DEVI void tc_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 
+DEVI void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// Each thread of the warp writes 32 consecutive 32-bit columns of its own TMEM lane.
+DEVI void tc_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
+        "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+        "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major operand tile stored as rows of
 // 128 bytes (64 bf16) with the 128-byte swizzle TMA produces: 8-row groups are
 // 1024 bytes apart (stride byte offset), version 1, layout SWIZZLE_128B.
@@ -221,10 +237,25 @@ DEVI uint64_t smem_desc_sw128(uint32_t saddr) {
     d |= (uint64_t)2 << 61;                          // SWIZZLE_128B
     return d;
 }
+// Descriptor for an MN-major operand (the N index contiguous) stored as blocks of
+// [K rows][64 bf16] with the 128-byte swizzle: K rows 128 bytes apart, 8-row
+// groups 1024 bytes apart (stride byte offset), the next 64-wide block of N
+// `mn_block_bytes` further on (leading byte offset).
+DEVI uint64_t smem_desc_sw128_mn(uint32_t saddr, uint32_t mn_block_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)((mn_block_bytes >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
 // Instruction descriptor, kind::f16: fp32 D, bf16 A and B, both K-major, M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// The same with B MN-major (bit 16: B transposed).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) { return idesc_bf16_f32(M, N) | (1u << 16); }
 
 // ---- legacy warp-level tensor core path (decode GEMV, flash attention) ----
 DEVI void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {

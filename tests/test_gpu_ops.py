@@ -79,6 +79,7 @@ ATTN_CASES = [
     (2, 64, 4, 4, [3, 0]),
     (1, 20, 32, 1, [0]),       # multi-query: 32 query heads share one KV head
     (2, 9, 24, 1, [3, 0]),
+    (1, 400, 8, 2, [100]),     # four 128-key tiles, a prompt continuing a cache
 ]
 
 
@@ -92,6 +93,33 @@ def test_flash_attention_prefill_matches_oracle(lib, B, T, H, Hk, pos0):
     L.llm_op_attention_prefill(q.to(DEV), kc.to(DEV), vc.to(DEV), p, out)
     torch.cuda.synchronize()
     # softmax weights and the output are rounded to bf16: |err| <= 3 * 2^-9 * max|v|.
+    err = np.abs(O.f64(out.cpu()) - ref)
+    assert err.max() <= 8e-3 * float(vc.abs().max()), err.max()
+
+
+def test_flash_attention_prefill_rescales_when_scores_grow(lib):
+    """Later keys score far higher than earlier ones (key norms growing along the
+    cache), so a row's running maximum grows by more than 2^8 between key tiles
+    and the accumulated output is rescaled in tensor memory."""
+    import llama_decoder_forward_fwd_b200 as L
+    B, T, H, Hk, d, S, pos0 = 1, 384, 8, 2, 128, 512, [0]
+    g = torch.Generator().manual_seed(21)
+    q = (torch.randn(B, T, H, d, generator=g) * 0.5).to(torch.bfloat16)
+    grow = (1.0 + torch.arange(S, dtype=torch.float32) / 16.0).view(1, 1, S, 1)
+    kc = (torch.randn(B, Hk, S, d, generator=g) * grow).to(torch.bfloat16)
+    vc = torch.randn(B, Hk, S, d, generator=g).to(torch.bfloat16)
+    ref = np.empty((B, T, H * d))
+    k = O.f64(kc[0, :, :T, :]).transpose(1, 0, 2)
+    v = O.f64(vc[0, :, :T, :]).transpose(1, 0, 2)
+    ref[0] = O.attention(O.f64(q[0]), k, v, np.arange(T), np.arange(T))
+    # the scores do grow by more than 2^8 (log2 domain) from the first key tile to the last
+    qf, kf = O.f64(q[0, :, 0]), O.f64(kc[0, 0, :T])
+    sc = qf @ kf.T / np.sqrt(d) * np.log2(np.e)
+    assert (sc[T - 1, 256:T].max() - sc[T - 1, :128].max()) > 8
+    out = torch.full((B, T, H * d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    p = torch.tensor(pos0, dtype=torch.int32, device=DEV)
+    L.llm_op_attention_prefill(q.to(DEV), kc.to(DEV), vc.to(DEV), p, out)
+    torch.cuda.synchronize()
     err = np.abs(O.f64(out.cpu()) - ref)
     assert err.max() <= 8e-3 * float(vc.abs().max()), err.max()
 
