@@ -17,12 +17,16 @@
 //              S = Q K^T (M = 128 rows, N = 128 keys, K = d) into one of two S
 //              accumulators, and O += P V (N = d, K = keys; V read MN-major, as it
 //              lies in the cache) into the O accumulator;
-//   warps 2-5  softmax, one thread per row (its TMEM lane): tcgen05.ld of the row
-//              of S, scale and causal mask, running maximum in the log2 domain,
-//              P = 2^(s - m) stored to shared memory in bf16 as the A operand of
-//              the PV product, running sum; at the end tcgen05.ld of O / sum.
-// The MMA thread issues S for tile j+2 as soon as P of tile j is written, so the
-// tensor cores compute the next scores while the softmax warps work.
+//   warps 2-9  softmax, two threads per row (its TMEM lane), 64 keys each:
+//              tcgen05.ld of the row of S, causal mask, the row's maximum (shared
+//              between the pair through shared memory), P = 2^(s - m) in the log2
+//              domain stored to shared memory in bf16 (two buffers) as the A operand
+//              of the PV product, partial sums; at the end tcgen05.ld of O / sum.
+// The MMA thread issues S for tile j+2 as soon as P of tile j is written, and the
+// softmax of tile j+1 does not wait for PV of tile j (unless O must be rescaled),
+// so the tensor cores and the softmax warps work at the same time.
+// CTAs are numbered longest row block first across all (sequence, KV head)
+// pairs, so the first wave takes the longest causal rows.
 // O is rescaled (tcgen05.ld, scale, tcgen05.st) only when a row's maximum grows
 // by more than 2^8 over the maximum its P values were taken against (the
 // conditional rescaling of FlashAttention-4): P stays below 256, exact in the
@@ -34,16 +38,38 @@
 
 namespace lfw {
 
-constexpr int FA_THREADS = 192;
+constexpr int FA_THREADS = 320;
 constexpr int FA_ROWS = 128;
 constexpr int FA_KT = 128;                      // keys per tile
 constexpr int FA_D = 128;
 constexpr int FA_HALF = 128 * 128;              // [128 rows][64 bf16]: 16 KB
 constexpr int FA_TILE = 2 * FA_HALF;            // a K, V, Q or P tile: 32 KB
-constexpr int FA_SMEM = 1024 + 6 * FA_TILE + 256;
+constexpr int FA_SMEM = 1024 + 7 * FA_TILE + 128;  // K, V (2 stages each), Q, P (2 buffers), barriers
 constexpr uint32_t FA_TMEM_COLS = 512;          // S (2 x 128 columns), O (128)
 constexpr uint32_t FA_TMEM_O = 256;
 constexpr float FA_RESCALE_LOG2 = 8.f;
+
+// 2^x by the special-function unit (ex2.approx, flush-to-zero): relative error of
+// a few ulp, far below the bf16 rounding that P gets next; 2^-inf = +0.
+DEVI float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// 2^x on the FMA pipe, for a share of the elements so that the special-function
+// unit is not the only one computing exponentials: x = n + f with n the nearest
+// integer (added to the exponent field) and f in [-0.5, 0.5], 2^f by a cubic
+// fitted to minimise the relative error (at most 1.5e-4 in fp32 arithmetic, far
+// below the bf16 rounding P gets next). x is clamped at -126, so a masked score
+// gives 2^-126 instead of 0: nothing at the scale of the row's sum.
+DEVI float ex2_poly(float x) {
+    x = fmaxf(x, -126.f);
+    const float t = x + 12582912.f;       // 1.5 * 2^23: n lands in the low mantissa bits
+    const float f = x - (t - 12582912.f);
+    const float p = fmaf(fmaf(fmaf(0.05517166f, f, 0.24261114f), f, 0.69326097f), f, 0.99992806f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
 
 __global__ void __launch_bounds__(FA_THREADS, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -54,22 +80,28 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     uint8_t* Ks = smem;                  // 2 stages
     uint8_t* Vs = smem + 2 * FA_TILE;    // 2 stages
     uint8_t* Qs = smem + 4 * FA_TILE;
-    uint8_t* Ps = smem + 5 * FA_TILE;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 6 * FA_TILE);
+    uint8_t* Ps = smem + 5 * FA_TILE;    // 2 buffers
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 7 * FA_TILE);
     uint64_t* k_full = bars;
     uint64_t* k_empty = bars + 2;
     uint64_t* v_full = bars + 4;
     uint64_t* v_empty = bars + 6;
     uint64_t* s_full = bars + 8;
     uint64_t* p_full = bars + 10;
-    uint64_t* pv_done = bars + 11;
-    uint64_t* mma_done = bars + 12;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+    uint64_t* pv_done = bars + 12;
+    uint64_t* mma_done = bars + 14;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+    // [tile parity][half][row]: the pair's partial maxima, in fp16 (both threads take
+    // the maximum of the two rounded values, so they agree on it; the maximum only
+    // offsets the exponent)
+    __shared__ __half red_max[2][2][FA_ROWS];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.H / a.Hk;
-    const int rb = gridDim.x - 1 - blockIdx.x;  // longest rows first
-    const int b = blockIdx.y / a.Hk, kvh = blockIdx.y % a.Hk;
+    const int nbh = a.B * a.Hk;
+    const int nrb = gridDim.x / nbh;
+    const int rb = nrb - 1 - (int)blockIdx.x / nbh;  // longest row blocks first
+    const int b = (blockIdx.x % nbh) / a.Hk, kvh = blockIdx.x % a.Hk;
     uint32_t* err = a.err;
 
     if (warp == 0 && lane == 0) {
@@ -79,9 +111,9 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
             mbar_init(&v_full[i], 1);
             mbar_init(&v_empty[i], 1);
             mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], 256);
+            mbar_init(&pv_done[i], 1);
         }
-        mbar_init(p_full, 128);
-        mbar_init(pv_done, 1);
         mbar_init(mma_done, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tmK);
@@ -101,16 +133,44 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     const int nkt = p_max / FA_KT + 1;
     const long long kv_row0 = a.row_base + (long long)(b * a.Hk + kvh) * a.S_max;
 
+    // The producer issues the first two K and V tiles before helping to stage Q
+    // (the stages are free: nothing to wait for).
+    auto load_kv = [&](uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, int j) {
+        const int y = (int)(kv_row0 + (long long)j * FA_KT);
+        mbar_arrive_expect_tx(bar, FA_TILE);
+        for (int h = 0; h < 2; ++h)
+            for (int kb = 0; kb < 2; ++kb) tma_load_2d(dst + h * FA_HALF + kb * (FA_HALF / 2), tm, bar, h * 64, y + kb * 64);
+    };
+    if (warp == 0 && lane == 0) {
+        for (int j = 0; j < 2 && j < nkt; ++j) {
+            load_kv(Ks + j * FA_TILE, &tmK, &k_full[j], j);
+            load_kv(Vs + j * FA_TILE, &tmV, &v_full[j], j);
+        }
+    }
+
     // Stage this CTA's 128 query rows as the A operand of S = Q K^T: two 64-dim
-    // halves of [128 rows][128 bytes], 16-byte chunks XOR-swizzled by row.
-    for (int idx = threadIdx.x; idx < FA_ROWS * 16; idx += FA_THREADS) {
-        const int r = idx >> 4, c = idx & 15;
-        const int rg = row0 + r;
-        const int t = rg / G, h = kvh * G + (rg - t * G);
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (t < a.T)
-            v = *reinterpret_cast<const uint4*>(a.q + ((long long)(b * a.T + t) * a.H + h) * FA_D + c * 8);
-        *reinterpret_cast<uint4*>(Qs + (c >> 3) * FA_HALF + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v;
+    // halves of [128 rows][128 bytes], 16-byte chunks XOR-swizzled by row. Every
+    // load is issued before any is stored, so staging costs one memory round trip.
+    {
+        constexpr int QN = (FA_ROWS * 16 + FA_THREADS - 1) / FA_THREADS;
+        uint4 v[QN];
+#pragma unroll
+        for (int i = 0; i < QN; ++i) {
+            const int idx = threadIdx.x + i * FA_THREADS;
+            const int r = idx >> 4, c = idx & 15;
+            const int rg = row0 + r;
+            const int t = rg / G, h = kvh * G + (rg - t * G);
+            v[i] = make_uint4(0, 0, 0, 0);
+            if (idx < FA_ROWS * 16 && t < a.T)
+                v[i] = __ldcg(reinterpret_cast<const uint4*>(a.q + ((long long)(b * a.T + t) * a.H + h) * FA_D + c * 8));
+        }
+#pragma unroll
+        for (int i = 0; i < QN; ++i) {
+            const int idx = threadIdx.x + i * FA_THREADS;
+            const int r = idx >> 4, c = idx & 15;
+            if (idx < FA_ROWS * 16)
+                *reinterpret_cast<uint4*>(Qs + (c >> 3) * FA_HALF + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v[i];
+        }
     }
     fence_proxy_async();  // the tensor cores read Q through the async proxy
     tc_fence_before();
@@ -121,31 +181,23 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     if (warp == 0) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
-            int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};  // last tile loaded into each stage
+            // last tile loaded into each stage (tiles 0 and 1 went out above)
+            int last_k[2] = {nkt > 0 ? 0 : -1, nkt > 1 ? 1 : -1}, last_v[2] = {last_k[0], last_k[1]};
             bool ok = true;
-            for (int j = 0; j < nkt && ok; ++j) {
+            for (int j = 2; j < nkt && ok; ++j) {
                 const int st = j & 1;
                 const uint32_t ph = (j >> 1) & 1;
-                const int y = (int)(kv_row0 + (long long)j * FA_KT);
                 if (!mbar_wait(&k_empty[st], ph ^ 1u, err, DERR_ATTN_TMA_WAIT)) {
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(&k_full[st], FA_TILE);
-                for (int h = 0; h < 2; ++h)
-                    for (int kb = 0; kb < 2; ++kb)
-                        tma_load_2d(Ks + st * FA_TILE + h * FA_HALF + kb * (FA_HALF / 2), &tmK, &k_full[st], h * 64,
-                                    y + kb * 64);
+                load_kv(Ks + st * FA_TILE, &tmK, &k_full[st], j);
                 last_k[st] = j;
                 if (!mbar_wait(&v_empty[st], ph ^ 1u, err, DERR_ATTN_TMA_WAIT)) {
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(&v_full[st], FA_TILE);
-                for (int h = 0; h < 2; ++h)
-                    for (int kb = 0; kb < 2; ++kb)
-                        tma_load_2d(Vs + st * FA_TILE + h * FA_HALF + kb * (FA_HALF / 2), &tmV, &v_full[st], h * 64,
-                                    y + kb * 64);
+                load_kv(Vs + st * FA_TILE, &tmV, &v_full[st], j);
                 last_v[st] = j;
             }
             if (!ok) {
@@ -180,117 +232,131 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
             bool ok = issue_s(0);
             if (ok && nkt > 1) ok = issue_s(1);
             for (int j = 0; j < nkt && ok; ++j) {
-                const int st = j & 1;
-                if (!mbar_wait(p_full, j & 1, err, DERR_ATTN_MMA_WAIT)) break;
+                const int st = j & 1;  // K/V stage, S accumulator and P buffer of tile j
+                if (!mbar_wait(&p_full[st], (j >> 1) & 1, err, DERR_ATTN_MMA_WAIT)) break;
                 if (!mbar_wait(&v_full[st], (j >> 1) & 1, err, DERR_ATTN_MMA_WAIT)) break;
                 tc_fence_after();
-                const uint32_t va = smem_u32(Vs + st * FA_TILE);
+                const uint32_t va = smem_u32(Vs + st * FA_TILE), pj = pa + st * FA_TILE;
 #pragma unroll
                 for (int kk = 0; kk < FA_KT / 16; ++kk) {
                     // A = P: keys 16kk.. of the K-major P tile; B = V: the same 16 key rows,
                     // all 128 dims (the second 64-dim half FA_HALF bytes on)
-                    tc_mma_f16(tmem_base + FA_TMEM_O, smem_desc_sw128(pa + (kk >> 2) * FA_HALF + (kk & 3) * 32),
+                    tc_mma_f16(tmem_base + FA_TMEM_O, smem_desc_sw128(pj + (kk >> 2) * FA_HALF + (kk & 3) * 32),
                                smem_desc_sw128_mn(va + kk * 2048, FA_HALF), idO, (j | kk) != 0);
                 }
                 tc_commit(&v_empty[st]);
-                tc_commit(pv_done);
+                tc_commit(&pv_done[st]);
                 if (j + 2 < nkt) ok = issue_s(j + 2);
             }
             tc_commit(mma_done);  // arrives once every MMA issued above has completed
         }
     } else {
-        // ---------------- softmax (warps 2..5), one thread per row ----------------
-        const int q4 = warp & 3;  // the TMEM lane quarter this warp may access
+        // ---------------- softmax (warps 2..9): two threads per row ----------------
+        // Warps w and w+4 share TMEM lane quarter w % 4 (the rows); the first takes
+        // keys 0..63 of each tile, the second keys 64..127. They agree on the row's
+        // maximum through shared memory and keep their own partial sums.
+        const int q4 = warp & 3;             // the TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2;    // which 64 keys of a tile, and 64 dims of O
         const int r = q4 * 32 + lane;
         const int rg = row0 + r;
         const int t = rg / G, h = kvh * G + (rg - t * G);
         const int prow = t < a.T ? p0 + t : -1;
         const uint32_t lane_base = tmem_base + ((uint32_t)(q4 * 32) << 16);
         const float sl2 = a.scale_log2;
-        float m_used = -INFINITY, l = 0.f;
+        float m_used = -INFINITY, l = 0.f;   // m_used in the log2 domain
         bool ok = true;
-        uint8_t* prow_s = Ps + r * 128;
         for (int j = 0; j < nkt; ++j) {
             const int sb = j & 1;
             if (ok && !mbar_wait(&s_full[sb], (j >> 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
             tc_fence_after();
-            float s[FA_KT];
+            float s[64];
             {
-                uint32_t u[4][32];
+                uint32_t u[2][32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tc_ld_32x32b_x32(lane_base + sb * FA_KT + c * 32, u[c]);
+                for (int c = 0; c < 2; ++c) tc_ld_32x32b_x32(lane_base + sb * FA_KT + half * 64 + c * 32, u[c]);
                 tc_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
+                for (int c = 0; c < 2; ++c)
 #pragma unroll
                     for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(u[c][i]);
             }
-            const int key0 = j * FA_KT;
-            float mx = -INFINITY;
-            if (key0 + FA_KT - 1 <= prow) {
+            // raw maximum (the scale is positive), four independent chains
+            const int key0 = j * FA_KT + half * 64;
+            if (key0 + 63 > prow) {
 #pragma unroll
-                for (int i = 0; i < FA_KT; ++i) {
-                    s[i] *= sl2;
-                    mx = fmaxf(mx, s[i]);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < FA_KT; ++i) {
-                    s[i] = key0 + i <= prow ? s[i] * sl2 : -INFINITY;
-                    mx = fmaxf(mx, s[i]);
-                }
+                for (int i = 0; i < 64; ++i)
+                    if (key0 + i > prow) s[i] = -INFINITY;
             }
+            float mx4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+            for (int i = 4; i < 64; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], s[i]);
+            const __half mine = __float2half_ru(fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2);
+            red_max[sb][half][r] = mine;
+            named_bar_sync(1 + q4, 64);
+            const float mx = fmaxf(__half2float(mine), __half2float(red_max[sb][half ^ 1][r]));
             const float m_new = fmaxf(m_used, mx);
             const bool need = m_new > m_used + FA_RESCALE_LOG2;  // false while the row has seen no key
-            const float alpha = need ? exp2f(m_used - m_new) : 1.f;
-            if (j > 0) {
-                // PV of the previous tile has completed: O is stable and the P buffer free
-                if (ok && !mbar_wait(pv_done, (j - 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
+            const float alpha = need ? ex2_approx(m_used - m_new) : 1.f;
+            // P buffer sb is free once PV of tile j-2 has completed
+            if (j >= 2 && ok && !mbar_wait(&pv_done[sb], ((j - 2) >> 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
+                // rescale this thread's 64 dims of O: PV of tile j-1 has completed, PV of
+                // tile j waits for this P
+                const int pb = (j - 1) & 1;
+                if (ok && !mbar_wait(&pv_done[pb], ((j - 1) >> 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, need)) {
 #pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t u[32];
-                        tc_ld_32x32b_x32(lane_base + FA_TMEM_O + c * 32, u);
-                        tc_wait_ld();
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t u[32];
+                    tc_ld_32x32b_x32(lane_base + FA_TMEM_O + half * 64 + c * 32, u);
+                    tc_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-                        tc_st_32x32b_x32(lane_base + FA_TMEM_O + c * 32, u);
-                    }
-                    tc_wait_st();
+                    for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+                    tc_st_32x32b_x32(lane_base + FA_TMEM_O + half * 64 + c * 32, u);
                 }
+                tc_wait_st();
             }
             if (need) {
                 l *= alpha;
                 m_used = m_new;
             }
             const float muse = m_used == -INFINITY ? 0.f : m_used;
-            float sum = 0.f;
+            uint8_t* prow_s = Ps + sb * FA_TILE + half * FA_HALF + r * 128;
+            float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < FA_KT / 8; ++c) {
+            for (int c = 0; c < 8; ++c) {
                 float p[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    p[e] = exp2f(s[c * 8 + e] - muse);
-                    sum += p[e];
+                    // a quarter of the exponentials on the FMA pipe
+                    const float x = fmaf(s[c * 8 + e], sl2, -muse);
+                    p[e] = e < 6 ? ex2_approx(x) : ex2_poly(x);
+                    sum4[e & 3] += p[e];
                 }
                 const uint4 v = make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
                                            pack_bf16x2(p[6], p[7]));
-                *reinterpret_cast<uint4*>(prow_s + (c >> 3) * FA_HALF + (((c & 7) ^ (r & 7)) << 4)) = v;
+                *reinterpret_cast<uint4*>(prow_s + ((c ^ (r & 7)) << 4)) = v;
             }
-            l += sum;
+            l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
             fence_proxy_async();  // P is read by the tensor cores through the async proxy
             tc_fence_before();
-            mbar_arrive(p_full);
+            mbar_arrive(&p_full[sb]);
         }
-        if (ok && !mbar_wait(pv_done, (nkt - 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
+        // PV of the last tile (and so every earlier one) has completed
+        if (ok && !mbar_wait(&pv_done[(nkt - 1) & 1], ((nkt - 1) >> 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
         tc_fence_after();
+        // the row's sum is the two halves' sums (both taken against the same maximum),
+        // exchanged through the P buffers, which no MMA reads any more
+        float* red_l = reinterpret_cast<float*>(Ps);
+        red_l[half * FA_ROWS + r] = l;
+        named_bar_sync(1 + q4, 64);
+        l += red_l[(half ^ 1) * FA_ROWS + r];
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        __nv_bfloat16* dst = a.out + ((long long)(b * a.T + t) * a.H + h) * FA_D;
+        __nv_bfloat16* dst = a.out + ((long long)(b * a.T + t) * a.H + h) * FA_D + half * 64;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
             uint32_t u[32];
-            tc_ld_32x32b_x32(lane_base + FA_TMEM_O + c * 32, u);
+            tc_ld_32x32b_x32(lane_base + FA_TMEM_O + half * 64 + c * 32, u);
             tc_wait_ld();
             if (prow >= 0) {
 #pragma unroll
@@ -319,7 +385,9 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
 cudaError_t launch_attn_prefill(const AttnPrefillArgs& a, cudaStream_t s, bool pdl) {
     if (a.H % a.Hk != 0 || a.T < 1) return cudaErrorInvalidValue;
     const int G = a.H / a.Hk;
-    const dim3 grid((a.T * G + FA_ROWS - 1) / FA_ROWS, a.B * a.Hk);
+    const long long nblk = (long long)((a.T * G + FA_ROWS - 1) / FA_ROWS) * a.B * a.Hk;
+    if (nblk > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const dim3 grid((unsigned)nblk);
     cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM);
     if (e != cudaSuccess) return e;
     return launch_k(attn_prefill_kernel, grid, dim3(FA_THREADS), FA_SMEM, s, pdl, *a.tmK, *a.tmV, a);
