@@ -29,6 +29,13 @@
  *     unsupported shapes) are detected on the host before anything is queued.
  *   - Device-side waits are bounded; a wait that runs out sets the model's
  *     error word, which llm_synchronize() reports as LLM_ERR_DEVICE_TIMEOUT.
+ *   - The library also comes as a bounds-checking build (liblfwd_checked.so,
+ *     compiled with -DLLM_BOUNDS_CHECK, same entry points): before the accesses
+ *     whose indices come from run-time data (token ids, cache positions and
+ *     lengths) its kernels check them; a failed check skips the access and sets
+ *     the error word, which llm_synchronize() (or llm_op_synchronize() for the
+ *     single operations) reports as LLM_ERR_DEVICE_BOUNDS, naming the check.
+ *     The normal build compiles these checks out (it clamps token ids).
  */
 #ifndef LLAMA_FWD_H
 #define LLAMA_FWD_H
@@ -50,6 +57,11 @@ extern "C" {
 #define LLM_ERR_DEVICE_TIMEOUT  (-6)  /* a bounded device-side wait ran out */
 #define LLM_ERR_UNSUPPORTED     (-7)  /* valid request this build does not implement */
 #define LLM_ERR_BAD_ARG         (-8)  /* other invalid argument (e.g. a size) */
+#define LLM_ERR_DEVICE_BOUNDS   (-9)  /* a device-side index check failed
+                                         (bounds-checking build only) */
+
+/* ---- build flags (llm_build_flags) -------------------------------------- */
+#define LLM_BUILD_BOUNDS_CHECK  1   /* compiled with -DLLM_BOUNDS_CHECK */
 
 /* ---- element types ----------------------------------------------------- */
 #define LLM_F32   0   /* weights, activations and KV cache in fp32 */
@@ -226,8 +238,14 @@ int llm_kernel_times(llm_model* m, int n, double* total_ms, int64_t* launches, i
  */
 int llm_debug_wait_probe(llm_model* m, int which, double limit_ms);
 
-/* Wait for the model's stream; report a CUDA error or a device-side timeout. */
+/* Wait for the model's stream; report a CUDA error, a device-side timeout
+ * (LLM_ERR_DEVICE_TIMEOUT) or, in the bounds-checking build, a failed device
+ * index check (LLM_ERR_DEVICE_BOUNDS). Clears the model's error word. */
 int llm_synchronize(llm_model* m);
+
+/* LLM_BUILD_BOUNDS_CHECK if this library is the bounds-checking build, else 0.
+ * A host-only query: needs no GPU. */
+int llm_build_flags(void);
 
 /* Release everything the model allocated. NULL is accepted. */
 void llm_model_free(llm_model* m);
@@ -239,6 +257,12 @@ const char* llm_last_error(void);
  * Single-operation entry points. Each runs one of the model's kernels on
  * caller-provided device buffers, on `stream` (a cudaStream_t, NULL: default).
  * ==================================================================== */
+
+/* Wait for `stream` and report the single operations' device error word as
+ * llm_synchronize() does for a model (a device timeout or, in the
+ * bounds-checking build, a failed index check); clears the word. The word is
+ * shared by all single operations of the process. */
+int llm_op_synchronize(void* stream);
 
 /*
  * C = A B^T on the tensor cores (the prefill projection kernel, tcgen05/TMEM

@@ -13,7 +13,10 @@ from typing import Dict, List, Optional
 
 import torch
 
-from .build import LIB as LIB_PATH
+from .build import LIB as _LIB_PLAIN, LIB_CHECKED as _LIB_CHECKED
+
+# LLM_LIB_VARIANT=checked selects the bounds-checking build (liblfwd_checked.so).
+LIB_PATH = _LIB_CHECKED if os.environ.get("LLM_LIB_VARIANT") == "checked" else _LIB_PLAIN
 
 LLM_OK = 0
 LLM_ERR_BAD_CONFIG = -1
@@ -24,6 +27,8 @@ LLM_ERR_CUDA = -5
 LLM_ERR_DEVICE_TIMEOUT = -6
 LLM_ERR_UNSUPPORTED = -7
 LLM_ERR_BAD_ARG = -8
+LLM_ERR_DEVICE_BOUNDS = -9
+LLM_BUILD_BOUNDS_CHECK = 1
 LLM_F32 = 0
 LLM_BF16 = 1
 LLM_FLAG_CUDA_GRAPH = 1
@@ -72,6 +77,8 @@ _SIGS = {
     "llm_kernel_times": (_i, [_vp, _i, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), _i]),
     "llm_debug_wait_probe": (_i, [_vp, _i, ctypes.c_double]),
     "llm_synchronize": (_i, [_vp]),
+    "llm_build_flags": (_i, []),
+    "llm_op_synchronize": (_i, [_vp]),
     "llm_model_free": (None, [_vp]),
     "llm_last_error": (ctypes.c_char_p, []),
     "llm_op_gemm_bf16": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
@@ -189,6 +196,14 @@ def llm_debug_wait_probe(m, which: int, limit_ms: float):
 
 def llm_synchronize(m):
     check(load().llm_synchronize(m))
+
+
+def llm_build_flags() -> int:
+    return load().llm_build_flags()
+
+
+def llm_op_synchronize(stream=None):
+    check(load().llm_op_synchronize(_stream_ptr(stream)))
 
 
 def llm_model_free(m):

@@ -15,6 +15,7 @@
 // the streaming decode GEMV. With LLM_FLAG_PDL, launches use programmatic
 // dependent launch so a kernel's prologue overlaps the previous kernel's tail.
 #include "../../include/llama_fwd.h"
+#include "errors.cuh"
 #include "kernels.cuh"
 
 #include <math.h>
@@ -332,6 +333,7 @@ Epi base_epi(llm_model* m, int M, int T) {
     Epi e;
     e.M = M;
     e.T = T;
+    e.S_max = m->cfg.max_seq_len;
     e.err = m->d_err;
     return e;
 }
@@ -575,6 +577,7 @@ int run_embed(llm_model* m, const int32_t* tok, const float* h_in, int M) {
     ea.M = M;
     ea.D = m->cfg.dim;
     ea.vocab = m->cfg.vocab;
+    ea.err = m->d_err;
     KTimer timer(m, LLM_K_EMBED);
     CK(launch_embed(ea, m->bf16, m->stream, m->pdl));
     return LLM_OK;
@@ -1124,6 +1127,18 @@ int llm_debug_wait_probe(llm_model* m, int which, double limit_ms) {
     return LLM_OK;
 }
 
+// The status of a nonzero device error word (bounds-check codes carry their site).
+static int device_error(uint32_t err) {
+    if ((err & 0xFF000000u) == lfw::DERR_BOUNDS) {
+        static const char* site[] = {"?", "token id outside [0, vocab)", "KV-cache append position outside [0, max_seq_len)",
+                                     "RoPE table row outside [0, max_seq_len)", "attention over positions beyond the cache",
+                                     "cache length advanced past max_seq_len", "decode position outside [0, max_seq_len)"};
+        const uint32_t s = err & 0xFFu;
+        return fail(LLM_ERR_DEVICE_BOUNDS, "device bounds check failed: %s (code 0x%x)", site[s < 7 ? s : 0], err);
+    }
+    return fail(LLM_ERR_DEVICE_TIMEOUT, "device wait timed out (code 0x%x)", err);
+}
+
 int llm_synchronize(llm_model* m) {
     if (!m) return fail(LLM_ERR_NULL_PTR, "model is NULL");
     CK(cudaStreamSynchronize(m->stream));
@@ -1131,9 +1146,17 @@ int llm_synchronize(llm_model* m) {
     CK(cudaMemcpy(&err, m->d_err, 4, cudaMemcpyDeviceToHost));
     if (err) {
         cudaMemset(m->d_err, 0, 4);
-        return fail(LLM_ERR_DEVICE_TIMEOUT, "device wait timed out (code 0x%x)", err);
+        return device_error(err);
     }
     return LLM_OK;
+}
+
+int llm_build_flags(void) {
+#ifdef LLM_BOUNDS_CHECK
+    return LLM_BUILD_BOUNDS_CHECK;
+#else
+    return 0;
+#endif
 }
 
 // ---------------------------------------------------------------- single operations
@@ -1141,6 +1164,19 @@ static uint32_t* op_err_ptr() {
     uint32_t* p = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_op_err) != cudaSuccess) return nullptr;
     return p;
+}
+
+int llm_op_synchronize(void* stream) {
+    CK(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+    uint32_t* p = op_err_ptr();
+    if (!p) return fail(LLM_ERR_CUDA, "cudaGetSymbolAddress of the operations' error word failed");
+    uint32_t err = 0;
+    CK(cudaMemcpy(&err, p, 4, cudaMemcpyDeviceToHost));
+    if (err) {
+        cudaMemset(p, 0, 4);
+        return device_error(err);
+    }
+    return LLM_OK;
 }
 
 int llm_op_gemm_bf16(const void* A, const void* B, float* C, int M, int N, int K, void* stream) {

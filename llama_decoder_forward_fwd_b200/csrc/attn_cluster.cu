@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(AC_THREADS, 1)
     const int R = G - chunk * AC_RMAX < AC_RMAX ? G - chunk * AC_RMAX : AC_RMAX;
     const int head0 = kvh * G + chunk * AC_RMAX;  // first query head of the group
     int p0 = a.pos0[b];
+    if (threadIdx.x == 0) LFW_CHECK(p0 >= 0 && p0 < a.S_max, a.err, BC_ATTN_POS);
     p0 = p0 < 0 ? 0 : (p0 >= a.S_max ? a.S_max - 1 : p0);
     const int U = (p0 + AK) / AK;  // units covering keys 0 .. p0
     const int u0 = (int)((long long)rank * U / a.cs), u1 = (int)((long long)(rank + 1) * U / a.cs);

@@ -92,6 +92,7 @@ DEVI void attn_split_item(const AttnDecodeArgs& a, int split, int b, int kvh, in
     const KT* vc = reinterpret_cast<const KT*>(a.vc) + head_off;
 
     const int p0 = a.pos0[b];
+    if (threadIdx.x == 0) LFW_CHECK(p0 >= 0 && p0 + a.T <= a.S_max, a.err, BC_ATTN_POS);
     const int row0 = qc * R;
     const int t_last = min(a.T - 1, (row0 + R - 1) / G);
     // keys [0, limit) are visible to some row; never read past the cache

@@ -127,6 +127,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     pdl_trigger();
     pdl_wait();
     const int p0 = a.pos0[b];
+    if (threadIdx.x == 0) LFW_CHECK(p0 >= 0 && p0 + a.T <= a.S_max, err, BC_ATTN_POS);
     const int row0 = rb * FA_ROWS;
     const int t_last = min(a.T - 1, (row0 + FA_ROWS - 1) / G);
     const int p_max = min(p0 + t_last, a.S_max - 1);  // the last key any row of this CTA sees

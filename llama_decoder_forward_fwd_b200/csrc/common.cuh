@@ -9,29 +9,29 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "errors.cuh"
+
 #define DEVI __device__ __forceinline__
 
 namespace lfw {
 
-// Device error word codes (first one wins).
-enum : uint32_t {
-    DERR_NONE = 0,
-    DERR_GEMM_PRODUCER_WAIT = 0x101,
-    DERR_GEMM_MMA_WAIT = 0x102,
-    DERR_GEMM_EPI_WAIT = 0x103,
-    DERR_ATTN_TMA_WAIT = 0x201,
-    DERR_ATTN_MMA_WAIT = 0x202,
-    DERR_ATTN_SOFTMAX_WAIT = 0x203,
-    DERR_GEMV_PRODUCER_WAIT = 0x301,
-    DERR_GEMV_CONSUMER_WAIT = 0x302,
-    DERR_GRID_BARRIER_WAIT = 0x401,
-    DERR_MK_PRODUCER_WAIT = 0x402,
-    DERR_MK_CONSUMER_WAIT = 0x403,
-    DERR_PROBE_WAIT = 0x501,  // the wait probe (a wait that cannot complete)
-};
+// Bounds-checking build (-DLLM_BOUNDS_CHECK): LFW_CHECK(cond, err, site) records
+// a failed index check in the error word (first one wins) and yields false, so
+// the caller skips the access. In the normal build it is `true`, and the
+// condition is not evaluated.
+#ifdef LLM_BOUNDS_CHECK
+#define LFW_CHECK(cond, err, site) ::lfw::bounds_check((cond), (err), (site))
+#else
+#define LFW_CHECK(cond, err, site) true
+#endif
 
 // 4 seconds: far longer than any legitimate wait for one pipeline stage.
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
+
+DEVI bool bounds_check(bool ok, uint32_t* err, uint32_t site) {
+    if (!ok && err) atomicCAS(err, 0u, (uint32_t)DERR_BOUNDS | site);
+    return ok;
+}
 
 DEVI uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 

@@ -399,7 +399,10 @@ __global__ void __launch_bounds__(DS_THREADS, 1) decode_step_kernel(const Decode
         }
         fence_mbar_init();
     }
-    if (threadIdx.x < B) s_len[threadIdx.x] = a.seq_len[threadIdx.x];
+    if (threadIdx.x < B) {
+        s_len[threadIdx.x] = a.seq_len[threadIdx.x];
+        LFW_CHECK(s_len[threadIdx.x] >= 0 && s_len[threadIdx.x] < a.S_max, a.err, BC_DECODE_POS);
+    }
     __syncthreads();
     const AttnSplit asp = attn_split(s_len, B, a.Hk);
 

@@ -62,6 +62,7 @@ DEVI void epi_qkv_pair(const Epi& e, int m, int c, float v0, float v1) {
     const int Hd = e.H * e.d, Hkd = e.Hk * e.d;
     const int b = m / e.T;
     const int pos = e.pos0[b] + (m - b * e.T);
+    if (!LFW_CHECK(pos >= 0 && pos < e.S_max, e.err, BC_CACHE_POS)) return;
     if (c < Hd + Hkd) rope_pair(e, pos, c % e.d, v0, v1);
     if (c < Hd) {
         store2<AT>(reinterpret_cast<AT*>(e.q_out) + (long long)m * Hd + c, v0, v1);
@@ -81,6 +82,7 @@ DEVI void epi_qkv8(const Epi& e, int m, int c, float (&v)[8]) {
     const int Hd = e.H * e.d, Hkd = e.Hk * e.d;
     const int b = m / e.T;
     const int pos = e.pos0[b] + (m - b * e.T);
+    if (!LFW_CHECK(pos >= 0 && pos < e.S_max, e.err, BC_CACHE_POS)) return;
     if (c < Hd + Hkd) {
         const int ch = c % e.d;
 #pragma unroll

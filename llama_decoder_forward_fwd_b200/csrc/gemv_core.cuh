@@ -299,6 +299,7 @@ DEVI void gv_epi_prefetch(GvEpiOps<NB>& op, int tile, int N, int M, int m0, cons
                 } else if ((g & 1) == 0 && lr[q] < (e.H + e.Hk) * e.d) {
                     const int bq = mg / e.T;
                     const int pos = e.pos0[bq] + (mg - bq * e.T);
+                    if (!LFW_CHECK(pos >= 0 && pos < e.S_max, e.err, BC_ROPE_POS)) continue;
                     const long long ti = (long long)pos * (e.d >> 1) + ((lr[q] % e.d) >> 1);
                     op.a[n][h][q] = e.rope_cos[ti];
                     op.b[n][h][q] = e.rope_sin[ti];
@@ -314,6 +315,7 @@ DEVI void gv_qkv_pair(const Epi& e, int m, int col, float v0, float v1, float cs
     const int Hd = e.H * e.d, Hkd = e.Hk * e.d;
     const int b = m / e.T;
     const int pos = e.pos0[b] + (m - b * e.T);
+    if (!LFW_CHECK(pos >= 0 && pos < e.S_max, e.err, BC_CACHE_POS)) return;
     if (col < Hd + Hkd) {
         const float r0 = v0 * cs - v1 * sn;
         const float r1 = v0 * sn + v1 * cs;
@@ -456,7 +458,9 @@ DEVI void gv_epilogue(int tile, const float (&c)[NB / 8][4], int N, int M, int m
             if (lane < M) {
                 const unsigned long long k = __ldcg(ws.am_best + lane);
                 e.next_tok[lane] = am_key_index(k);
-                if (e.seq_len) e.seq_len[lane] += e.advance;
+                if (e.seq_len && LFW_CHECK(e.seq_len[lane] + e.advance <= e.S_max || e.S_max == 0, e.err,
+                                           BC_SEQ_ADVANCE))
+                    e.seq_len[lane] += e.advance;
                 ws.am_best[lane] = 0ull;
             }
             if (lane == 0) *ws.done_cnt = 0u;

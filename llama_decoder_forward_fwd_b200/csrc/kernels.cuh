@@ -259,6 +259,7 @@ struct EmbedArgs {
     const void* wnorm = nullptr;   // first layer's attention_norm
     float* ss = nullptr;           // [1][M]
     int M = 0, D = 0, vocab = 0;
+    uint32_t* err = nullptr;       // bounds-checking build: out-of-range token ids
 };
 cudaError_t launch_embed(const EmbedArgs& a, bool bf16, cudaStream_t s, bool pdl);
 // h_out = h; seq_len[b] += advance for b < B.

@@ -29,7 +29,8 @@ __global__ void __launch_bounds__(EMB_THREADS) embed_kernel(const EmbedArgs a) {
         hsrc = a.h_in + (long long)m * a.D;
     } else {
         int tok = a.tok[m];
-        tok = tok < 0 ? 0 : (tok >= a.vocab ? a.vocab - 1 : tok);
+        if (threadIdx.x == 0) LFW_CHECK(tok >= 0 && tok < a.vocab, a.err, BC_TOKEN);
+        tok = tok < 0 ? 0 : (tok >= a.vocab ? a.vocab - 1 : tok);  // never read outside the table
         src = reinterpret_cast<const WT*>(a.E) + (long long)tok * a.D;
     }
     float ss = 0.f;

@@ -42,6 +42,18 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, name), name
 
 
+def test_bounds_checking_build_loads_with_the_same_symbols(lib):
+    """The -DLLM_BOUNDS_CHECK build exports the same calls and says what it is
+    (llm_build_flags is a host-only query)."""
+    B.build()
+    checked = ctypes.CDLL(B.LIB_CHECKED)
+    for name in declared_functions():
+        assert hasattr(checked, name), name
+    checked.llm_build_flags.restype = ctypes.c_int
+    assert checked.llm_build_flags() == L.LLM_BUILD_BOUNDS_CHECK
+    assert lib.llm_build_flags() == 0
+
+
 def test_binding_covers_every_declared_symbol():
     assert sorted(L.exported_symbols()) == declared_functions()
 
