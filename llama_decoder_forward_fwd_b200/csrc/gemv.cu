@@ -59,10 +59,12 @@ DEVI void logits_finish(const Epi& e, int M, int ntiles, int* last_s) {
 // cooperative (every CTA resident), so a row tile split over several CTAs is
 // finished by its first CTA, which waits for the other CTAs' pieces; they publish
 // them as soon as they reach the end of their part and move on.
-// Ring depth: 5 stages for the layer projections; the lm_head,
-// one long stream of 1 GB, keeps 10 stages in flight (measured: 163 against
-// 172 us at the Llama-3-8B vocabulary), which the layer projections do not gain from.
-template <int EPI> constexpr int gv_stages() { return EPI == EPI_LOGITS ? 10 : 5; }
+// Ring depth: 8 stages (128 KB) for the layer projections, about the bytes an SM
+// has in flight at its share of HBM bandwidth under load (measured at the
+// Llama-3-8B shape: 3.51 ms per decode token against 3.58 with 5 stages, 3.51 with
+// 7 or 9, 3.57 with 10); the lm_head, one long stream of 1 GB, keeps 10 stages
+// (163 against 172 us with 5).
+template <int EPI> constexpr int gv_stages() { return EPI == EPI_LOGITS ? 10 : 8; }
 constexpr int GV_THREADS = GV_CONSUMERS + 32;   // 8 consumer warps + 1 producer warp
 constexpr int GV_XS_BYTES = 56 * 1024 + 256;    // token rows staged whole when they fit (one token's
                                                 // split rows of the 14336-wide FFN input)
