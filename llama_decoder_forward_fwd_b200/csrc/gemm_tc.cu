@@ -3,7 +3,7 @@
 // llama3 from scratch": q_per_token = x @ wq_head^T, here for all tokens and all
 // heads at once), fp32 accumulation in tensor memory.
 //
-// Persistent kernel, one CTA per SM, 6 warps:
+// Persistent kernel, one CTA per SM, 10 warps:
 //   warp 0     TMA producer: streams 128x64 A tiles and 256x64 B tiles into a
 //              4-stage shared-memory ring (128-byte swizzle), one mbarrier per
 //              stage for "full" (transaction bytes) and one for "empty".
@@ -11,10 +11,11 @@
 //              K=16; four per 64-wide k block) from one elected thread into one
 //              of two 256-column accumulators, committing "empty" per stage and
 //              "accumulator full" per tile.
-//   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter (rows) of the
-//              accumulator, the fused epilogue (RMSNorm scale, RoPE + KV-cache
-//              append, SwiGLU, or residual add) and stores; then release the
-//              accumulator so the MMA warp can start the tile after next.
+//   warps 2-9  epilogue, two warps per 32-lane quarter (rows) of the accumulator,
+//              each half of the columns: tcgen05.ld, the fused epilogue (RMSNorm
+//              scale, RoPE + KV-cache append, SwiGLU, or residual add) and stores,
+//              with each chunk's global operands loaded a chunk ahead; then release
+//              the accumulator so the MMA warp can start the tile after next.
 // Tiles are visited m-fastest so CTAs running together share weight tiles in L2.
 #include "epilogue.cuh"
 
@@ -25,7 +26,7 @@ constexpr int G_A_BYTES = GEMM_BM * GEMM_BK * 2;  // 16 KB
 constexpr int G_B_BYTES = GEMM_BN * GEMM_BK * 2;  // 32 KB
 constexpr int G_STAGE_BYTES = G_A_BYTES + G_B_BYTES;
 constexpr int G_SMEM_BYTES = G_STAGES * G_STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-constexpr int G_THREADS = 192;
+constexpr int G_THREADS = 320;
 constexpr uint32_t G_TMEM_COLS = 512;
 
 struct GemmKernelParams {
@@ -49,6 +50,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint32_t* err = p.epi.err;
+    __shared__ float ss_half[2][GEMM_BM];  // residual epilogue: the row sums of squares of the two halves
 
     if (warp == 0 && lane == 0) {
         for (int i = 0; i < G_STAGES; ++i) {
@@ -57,7 +59,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
-            mbar_init(&tempty[i], 4);
+            mbar_init(&tempty[i], 8);
         }
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
@@ -170,25 +172,70 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             }
         }
     } else {
-        // ---------------- epilogue (warps 2..5) ----------------
+        // ---------------- epilogue (warps 2..9) ----------------
+        // Warps w and w+4 share TMEM lane quarter w % 4 (32 rows of the tile); the
+        // first takes the tile's first 128 columns, the second the last 128 (for
+        // SwiGLU: the first and last two 32-column chunks of the w1 and w3 halves).
+        // The global operands of a chunk (residual h and norm weights, RoPE cos/sin)
+        // and the row's RMSNorm scale are loaded one chunk ahead, the first ones
+        // before the accumulator is waited for, so the stores do not wait on them.
         const int quarter = warp & 3;  // TMEM lanes this warp may access
+        const int half = (warp - 2) >> 2;
         const int row_in_tile = quarter * 32 + lane;
         const Epi& e = p.epi;
+        constexpr int NCH = EPI == EPI_SWIGLU ? 2 : 4;  // 32-column chunks per warp
+        // After a failed (timed-out) wait a warp stops waiting but keeps walking the
+        // tiles, so the two warps of a lane quarter always meet at their named barriers.
+        bool ok = true;
         int it = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
             const int mb = tile % num_m, nb = tile / num_m;
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
-            if (!mbar_wait(&tfull[acc], acc_phase, err, DERR_GEMM_EPI_WAIT)) break;
-            tc_fence_after();
             const int m = mb * GEMM_BM + row_in_tile;
             const bool valid = m < p.M;
             const float rinv = valid ? row_rinv(e.norm, m) : 0.f;
+            // operands of chunk ch: columns c0(ch) .. c0(ch)+31
+            auto col0 = [&](int ch) { return nb * GEMM_BN + half * (GEMM_BN / 2) + ch * 32; };
+            float4 opa[8], opb[8];  // RESID: h (8 float4) and norm weights (4 uint4 in opb[0..3]);
+                                    // QKV: cos (opa[0..3]) and sin (opb[0..3]) of the chunk's 16 pairs
+            auto load_ops = [&](int ch) {
+                if (!valid) return;
+                const int c0 = col0(ch);
+                if (EPI == EPI_RESID) {
+                    const float4* hp = reinterpret_cast<const float4*>(e.h + (size_t)m * e.D + c0);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) opa[i] = hp[i];
+                    const float4* wp = reinterpret_cast<const float4*>(reinterpret_cast<const __nv_bfloat16*>(e.wnext) + c0);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) opb[i] = wp[i];
+                } else if (EPI == EPI_QKV_ROPE) {
+                    const int Hd = e.H * e.d, Hkd = e.Hk * e.d;
+                    if (c0 < Hd + Hkd) {
+                        const int b = m / e.T;
+                        const int pos = e.pos0[b] + (m - b * e.T);
+                        if (pos >= 0 && pos < e.S_max) {
+                            const long long ti = (long long)pos * (e.d >> 1) + ((c0 % e.d) >> 1);
+                            const float4* cp = reinterpret_cast<const float4*>(e.rope_cos + ti);
+                            const float4* sp = reinterpret_cast<const float4*>(e.rope_sin + ti);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                opa[i] = cp[i];
+                                opb[i] = sp[i];
+                            }
+                        }
+                    }
+                }
+            };
+            if (EPI == EPI_RESID || EPI == EPI_QKV_ROPE) load_ops(0);
+            if (ok && !mbar_wait(&tfull[acc], acc_phase, err, DERR_GEMM_EPI_WAIT)) ok = false;
+            tc_fence_after();
             const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * GEMM_BN;
             if (EPI == EPI_SWIGLU) {
                 const int n0 = nb * (GEMM_BN / 2);
 #pragma unroll 1
-                for (int ch = 0; ch < 4; ++ch) {
+                for (int cc = 0; cc < NCH; ++cc) {
+                    const int ch = half * NCH + cc;
                     uint32_t ra[32], rc[32];
                     tc_ld_32x32b_x32(tbase + ch * 32, ra);
                     tc_ld_32x32b_x32(tbase + GEMM_BN / 2 + ch * 32, rc);
@@ -208,12 +255,20 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             } else {
                 float ss = 0.f;
 #pragma unroll 1
-                for (int ch = 0; ch < GEMM_BN / 32; ++ch) {
+                for (int cc = 0; cc < NCH; ++cc) {
                     uint32_t r[32];
-                    tc_ld_32x32b_x32(tbase + ch * 32, r);
+                    tc_ld_32x32b_x32(tbase + half * (GEMM_BN / 2) + cc * 32, r);
+                    // this chunk's operands are in opa/opb; fetch the next chunk's while
+                    // the accumulator values arrive
+                    float4 ca[8], cb[4];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) ca[i] = opa[i];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) cb[i] = opb[i];
+                    if ((EPI == EPI_RESID || EPI == EPI_QKV_ROPE) && cc + 1 < NCH) load_ops(cc + 1);
                     tc_wait_ld();
                     if (!valid) continue;
-                    const int c0 = nb * GEMM_BN + ch * 32;
+                    const int c0 = col0(cc);
 #pragma unroll
                     for (int j = 0; j < 32; j += 8) {
                         float v[8];
@@ -222,16 +277,41 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                         if (EPI == EPI_STORE_F32) {
                             store8<float>(e.y + (size_t)m * e.ldy + c0 + j, v);
                         } else if (EPI == EPI_QKV_ROPE) {
-                            epi_qkv8<__nv_bfloat16>(e, m, c0 + j, v);
+                            const int Hd = e.H * e.d, Hkd = e.Hk * e.d;
+                            const int c = c0 + j;
+                            const int b = m / e.T;
+                            const int pos = e.pos0[b] + (m - b * e.T);
+                            if (!LFW_CHECK(pos >= 0 && pos < e.S_max, e.err, BC_CACHE_POS)) continue;
+                            if (c < Hd + Hkd) {
+                                // pairs 4j/8 .. of the chunk: cos/sin elements j/2 .. j/2+3
+                                const float4 cs = ca[j >> 3], sn = cb[j >> 3];
+                                const float cv[4] = {cs.x, cs.y, cs.z, cs.w}, sv[4] = {sn.x, sn.y, sn.z, sn.w};
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    const float x0 = v[2 * q], x1 = v[2 * q + 1];
+                                    v[2 * q] = x0 * cv[q] - x1 * sv[q];
+                                    v[2 * q + 1] = x0 * sv[q] + x1 * cv[q];
+                                }
+                            }
+                            if (c < Hd) {
+                                store8<__nv_bfloat16>(reinterpret_cast<__nv_bfloat16*>(e.q_out) + (size_t)m * Hd + c, v);
+                            } else {
+                                int kc = c - Hd;
+                                const bool isv = kc >= Hkd;
+                                if (isv) kc -= Hkd;
+                                const int kvh = kc / e.d, dd = kc - kvh * e.d;
+                                __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(isv ? e.v_cache : e.k_cache);
+                                store8<__nv_bfloat16>(base + ((long long)(b * e.Hk + kvh) * e.S_max + pos) * e.d + dd, v);
+                            }
                         } else if (EPI == EPI_RESID) {
                             float* hp = e.h + (size_t)m * e.D + c0 + j;
-                            const float4 h0 = reinterpret_cast<const float4*>(hp)[0];
-                            const float4 h1 = reinterpret_cast<const float4*>(hp)[1];
+                            const float4 h0 = ca[j >> 2], h1 = ca[(j >> 2) + 1];
                             float hn[8] = {h0.x + v[0], h0.y + v[1], h0.z + v[2], h0.w + v[3],
                                            h1.x + v[4], h1.y + v[5], h1.z + v[6], h1.w + v[7]};
                             store8<float>(hp, hn);
-                            const uint4 wv = *reinterpret_cast<const uint4*>(
-                                reinterpret_cast<const __nv_bfloat16*>(e.wnext) + c0 + j);
+                            const float4 wf = cb[j >> 3];
+                            const uint4 wv = make_uint4(__float_as_uint(wf.x), __float_as_uint(wf.y),
+                                                        __float_as_uint(wf.z), __float_as_uint(wf.w));
                             float hw[8];
                             hw[0] = hn[0] * bf16lo(wv.x);
                             hw[1] = hn[1] * bf16hi(wv.x);
@@ -248,7 +328,15 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                         }
                     }
                 }
-                if (EPI == EPI_RESID && valid) e.ss_out[(size_t)nb * e.ss_out_ld + m] = ss;
+                if (EPI == EPI_RESID) {
+                    // the row's sum of squares over the tile: the two halves' sums, added
+                    // in a fixed order
+                    ss_half[half][row_in_tile] = ss;
+                    named_bar_sync(1 + quarter, 64);
+                    if (half == 0 && valid)
+                        e.ss_out[(size_t)nb * e.ss_out_ld + m] = ss + ss_half[1][row_in_tile];
+                    named_bar_sync(1 + quarter, 64);  // the slots are rewritten by the next tile
+                }
             }
             tc_fence_before();
             __syncwarp();
