@@ -7,10 +7,13 @@
 // j <= p of KV head h / G (G = n_heads / n_kv_heads), future keys masked, softmax,
 // weighted sum of values, heads concatenated.
 //
-// Layout of the work. A CTA owns 128 "rows" of one (sequence, KV head): row r is
-// (token t = r / G, query head kvh*G + r % G), so the G query heads that share a
-// KV head sit in one CTA and every K/V tile is loaded once for all of them.
-// Keys go in tiles of 128, d = 128. Six warps:
+// Layout of the work. A work item is 128 "rows" of one (sequence, KV head): row r
+// is (token t = r / G, query head kvh*G + r % G), so the G query heads that share a
+// KV head sit together and every K/V tile is loaded once for all of them. The
+// kernel is persistent (one CTA per SM, TMEM allocated once): each CTA runs a
+// fixed sequence of items, longest causal rows first, and every role walks the
+// same sequence, so the barrier phases follow one running tile count. Keys go in
+// tiles of 128, d = 128. Ten warps:
 //   warp 0     TMA producer: K and V tiles (two 64-dim halves, 128-byte swizzle)
 //              from the KV cache into 2-stage rings, K and V on their own barriers;
 //   warp 1     allocates 512 TMEM columns and issues tcgen05.mma from one thread:
@@ -25,8 +28,10 @@
 // The MMA thread issues S for tile j+2 as soon as P of tile j is written, and the
 // softmax of tile j+1 does not wait for PV of tile j (unless O must be rescaled),
 // so the tensor cores and the softmax warps work at the same time.
-// CTAs are numbered longest row block first across all (sequence, KV head)
-// pairs, so the first wave takes the longest causal rows.
+// The softmax warps stage the next item's query rows as soon as the current item's
+// last S product is complete (in the swizzled layout, one memory round trip), so
+// the MMA thread starts the next item's S products while they finish the last
+// tile and write out O.
 // O is rescaled (tcgen05.ld, scale, tcgen05.st) only when a row's maximum grows
 // by more than 2^8 over the maximum its P values were taken against (the
 // conditional rescaling of FlashAttention-4): P stays below 256, exact in the
@@ -44,9 +49,10 @@ constexpr int FA_KT = 128;                      // keys per tile
 constexpr int FA_D = 128;
 constexpr int FA_HALF = 128 * 128;              // [128 rows][64 bf16]: 16 KB
 constexpr int FA_TILE = 2 * FA_HALF;            // a K, V, Q or P tile: 32 KB
-constexpr int FA_SMEM = 1024 + 7 * FA_TILE + 128;  // K, V (2 stages each), Q, P (2 buffers), barriers
+constexpr int FA_SMEM = 1024 + 7 * FA_TILE + 256;  // K, V (2 stages each), Q, P (2 buffers), barriers
 constexpr uint32_t FA_TMEM_COLS = 512;          // S (2 x 128 columns), O (128)
 constexpr uint32_t FA_TMEM_O = 256;
+constexpr uint32_t FA_TMEM_L = 384;             // two columns: the row sums of the pair's halves
 constexpr float FA_RESCALE_LOG2 = 8.f;
 
 // 2^x by the special-function unit (ex2.approx, flush-to-zero): relative error of
@@ -71,6 +77,22 @@ DEVI float ex2_poly(float x) {
     return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// tcgen05.st / tcgen05.ld of one 32-bit column of this thread's TMEM lane.
+DEVI void tc_st_x1(uint32_t taddr, uint32_t v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
+DEVI uint32_t tc_ld_x1(uint32_t taddr) {
+    uint32_t v;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v) : "r"(taddr) : "memory");
+    return v;
+}
+
+// A work item: the 128 rows of one (sequence, KV head) starting at row0.
+struct FaItem {
+    int b, kvh, row0, p0, nkt;
+    long long kv_row0;  // cache row of this (sequence, KV head)'s position 0
+};
+
 __global__ void __launch_bounds__(FA_THREADS, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const AttnPrefillArgs a) {
@@ -89,8 +111,9 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     uint64_t* s_full = bars + 8;
     uint64_t* p_full = bars + 10;
     uint64_t* pv_done = bars + 12;
-    uint64_t* mma_done = bars + 14;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+    uint64_t* q_full = bars + 14;    // the next item's Q is staged (items after the first)
+    uint64_t* mma_done = bars + 15;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
     // [tile parity][half][row]: the pair's partial maxima, in fp16 (both threads take
     // the maximum of the two rounded values, so they agree on it; the maximum only
     // offsets the exponent)
@@ -99,10 +122,62 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.H / a.Hk;
     const int nbh = a.B * a.Hk;
-    const int nrb = gridDim.x / nbh;
-    const int rb = nrb - 1 - (int)blockIdx.x / nbh;  // longest row blocks first
-    const int b = (blockIdx.x % nbh) / a.Hk, kvh = blockIdx.x % a.Hk;
+    const int nrb = (a.T * G + FA_ROWS - 1) / FA_ROWS;
+    const int total = nrb * nbh;
     uint32_t* err = a.err;
+
+    // Items are numbered longest causal rows first (item k: row block nrb-1-k/nbh of
+    // (sequence, KV head) k % nbh); CTA c takes items c, 2g-1-c, 2g+c, ... (g CTAs),
+    // which balances the rows' lengths over the CTAs.
+    auto item_of = [&](int ki) -> int {
+        const int k = ki * (int)gridDim.x + ((ki & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+        return k < total ? k : -1;
+    };
+    auto describe = [&](int k) -> FaItem {
+        FaItem it;
+        const int bh = k % nbh;
+        it.b = bh / a.Hk;
+        it.kvh = bh % a.Hk;
+        it.row0 = (nrb - 1 - k / nbh) * FA_ROWS;
+        it.p0 = a.pos0[it.b];
+        const int t_last = min(a.T - 1, (it.row0 + FA_ROWS - 1) / G);
+        const int p_max = min(it.p0 + t_last, a.S_max - 1);  // the last key any row of the item sees
+        it.nkt = max(p_max, 0) / FA_KT + 1;
+        it.kv_row0 = a.row_base + (long long)(it.b * a.Hk + it.kvh) * a.S_max;
+        return it;
+    };
+    auto load_kv = [&](uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, long long kv_row0, int j) {
+        const int y = (int)(kv_row0 + (long long)j * FA_KT);
+        mbar_arrive_expect_tx(bar, FA_TILE);
+        for (int h = 0; h < 2; ++h)
+            for (int kb = 0; kb < 2; ++kb) tma_load_2d(dst + h * FA_HALF + kb * (FA_HALF / 2), tm, bar, h * 64, y + kb * 64);
+    };
+    // Stage an item's 128 query rows as the A operand of S = Q K^T: two 64-dim
+    // halves of [128 rows][128 bytes], 16-byte chunks XOR-swizzled by row; 16 loads
+    // per thread are in flight before any is stored.
+    auto stage_q = [&](const FaItem& it, int tid, int nthr) {
+        constexpr int QB = 16;
+        for (int base = tid; base < FA_ROWS * 16; base += nthr * QB) {
+            uint4 v[QB];
+#pragma unroll
+            for (int i = 0; i < QB; ++i) {
+                const int idx = base + i * nthr;
+                const int r = idx >> 4, c = idx & 15;
+                const int rg = it.row0 + r;
+                const int t = rg / G, h = it.kvh * G + (rg - t * G);
+                v[i] = make_uint4(0, 0, 0, 0);
+                if (idx < FA_ROWS * 16 && t < a.T)
+                    v[i] = __ldcg(reinterpret_cast<const uint4*>(a.q + ((long long)(it.b * a.T + t) * a.H + h) * FA_D + c * 8));
+            }
+#pragma unroll
+            for (int i = 0; i < QB; ++i) {
+                const int idx = base + i * nthr;
+                const int r = idx >> 4, c = idx & 15;
+                if (idx < FA_ROWS * 16)
+                    *reinterpret_cast<uint4*>(Qs + (c >> 3) * FA_HALF + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v[i];
+            }
+        }
+    };
 
     if (warp == 0 && lane == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -114,6 +189,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
             mbar_init(&p_full[i], 256);
             mbar_init(&pv_done[i], 1);
         }
+        mbar_init(q_full, 256);
         mbar_init(mma_done, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tmK);
@@ -126,53 +202,16 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
 
     pdl_trigger();
     pdl_wait();
-    const int p0 = a.pos0[b];
-    if (threadIdx.x == 0) LFW_CHECK(p0 >= 0 && p0 + a.T <= a.S_max, err, BC_ATTN_POS);
-    const int row0 = rb * FA_ROWS;
-    const int t_last = min(a.T - 1, (row0 + FA_ROWS - 1) / G);
-    const int p_max = min(p0 + t_last, a.S_max - 1);  // the last key any row of this CTA sees
-    const int nkt = p_max / FA_KT + 1;
-    const long long kv_row0 = a.row_base + (long long)(b * a.Hk + kvh) * a.S_max;
-
-    // The producer issues the first two K and V tiles before helping to stage Q
-    // (the stages are free: nothing to wait for).
-    auto load_kv = [&](uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, int j) {
-        const int y = (int)(kv_row0 + (long long)j * FA_KT);
-        mbar_arrive_expect_tx(bar, FA_TILE);
-        for (int h = 0; h < 2; ++h)
-            for (int kb = 0; kb < 2; ++kb) tma_load_2d(dst + h * FA_HALF + kb * (FA_HALF / 2), tm, bar, h * 64, y + kb * 64);
-    };
+    // The first item: the producer issues its first two K and V tiles (the stages are
+    // free), then every thread helps to stage its Q.
+    const FaItem it0 = describe(item_of(0));  // the grid never exceeds the items
     if (warp == 0 && lane == 0) {
-        for (int j = 0; j < 2 && j < nkt; ++j) {
-            load_kv(Ks + j * FA_TILE, &tmK, &k_full[j], j);
-            load_kv(Vs + j * FA_TILE, &tmV, &v_full[j], j);
+        for (int j = 0; j < 2 && j < it0.nkt; ++j) {
+            load_kv(Ks + j * FA_TILE, &tmK, &k_full[j], it0.kv_row0, j);
+            load_kv(Vs + j * FA_TILE, &tmV, &v_full[j], it0.kv_row0, j);
         }
     }
-
-    // Stage this CTA's 128 query rows as the A operand of S = Q K^T: two 64-dim
-    // halves of [128 rows][128 bytes], 16-byte chunks XOR-swizzled by row. Every
-    // load is issued before any is stored, so staging costs one memory round trip.
-    {
-        constexpr int QN = (FA_ROWS * 16 + FA_THREADS - 1) / FA_THREADS;
-        uint4 v[QN];
-#pragma unroll
-        for (int i = 0; i < QN; ++i) {
-            const int idx = threadIdx.x + i * FA_THREADS;
-            const int r = idx >> 4, c = idx & 15;
-            const int rg = row0 + r;
-            const int t = rg / G, h = kvh * G + (rg - t * G);
-            v[i] = make_uint4(0, 0, 0, 0);
-            if (idx < FA_ROWS * 16 && t < a.T)
-                v[i] = __ldcg(reinterpret_cast<const uint4*>(a.q + ((long long)(b * a.T + t) * a.H + h) * FA_D + c * 8));
-        }
-#pragma unroll
-        for (int i = 0; i < QN; ++i) {
-            const int idx = threadIdx.x + i * FA_THREADS;
-            const int r = idx >> 4, c = idx & 15;
-            if (idx < FA_ROWS * 16)
-                *reinterpret_cast<uint4*>(Qs + (c >> 3) * FA_HALF + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = v[i];
-        }
-    }
+    stage_q(it0, threadIdx.x, FA_THREADS);
     fence_proxy_async();  // the tensor cores read Q through the async proxy
     tc_fence_before();
     __syncthreads();
@@ -180,33 +219,43 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        // ---------------- TMA producer ----------------
-        if (lane == 0) {
-            // last tile loaded into each stage (tiles 0 and 1 went out above)
-            int last_k[2] = {nkt > 0 ? 0 : -1, nkt > 1 ? 1 : -1}, last_v[2] = {last_k[0], last_k[1]};
-            bool ok = true;
-            for (int j = 2; j < nkt && ok; ++j) {
-                const int st = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
-                if (!mbar_wait(&k_empty[st], ph ^ 1u, err, DERR_ATTN_TMA_WAIT)) {
-                    ok = false;
-                    break;
+        // ---------------- producer: Q of each later item, K and V tiles ----------------
+        int last_k[2] = {it0.nkt > 0 ? 0 : -1, it0.nkt > 1 ? 1 : -1};  // last running tile loaded per stage
+        int last_v[2] = {last_k[0], last_k[1]};
+        bool ok = true;
+        int g = 0;  // running tile index over this CTA's items
+        for (int ki = 0; ok; ++ki) {
+            const int k = item_of(ki);
+            if (k < 0) break;
+            const FaItem it = describe(k);
+            if (lane == 0) (void)LFW_CHECK(it.p0 >= 0 && it.p0 + a.T <= a.S_max, err, BC_ATTN_POS);
+            const int j0 = ki == 0 ? min(2, it.nkt) : 0;
+            if (lane == 0) {
+                for (int j = j0; j < it.nkt && ok; ++j) {
+                    const int gg = g + j, st = gg & 1;
+                    const uint32_t ph = (gg >> 1) & 1;
+                    if (!mbar_wait(&k_empty[st], ph ^ 1u, err, DERR_ATTN_TMA_WAIT)) {
+                        ok = false;
+                        break;
+                    }
+                    load_kv(Ks + st * FA_TILE, &tmK, &k_full[st], it.kv_row0, j);
+                    last_k[st] = gg;
+                    if (!mbar_wait(&v_empty[st], ph ^ 1u, err, DERR_ATTN_TMA_WAIT)) {
+                        ok = false;
+                        break;
+                    }
+                    load_kv(Vs + st * FA_TILE, &tmV, &v_full[st], it.kv_row0, j);
+                    last_v[st] = gg;
                 }
-                load_kv(Ks + st * FA_TILE, &tmK, &k_full[st], j);
-                last_k[st] = j;
-                if (!mbar_wait(&v_empty[st], ph ^ 1u, err, DERR_ATTN_TMA_WAIT)) {
-                    ok = false;
-                    break;
-                }
-                load_kv(Vs + st * FA_TILE, &tmV, &v_full[st], j);
-                last_v[st] = j;
             }
-            if (!ok) {
-                // let copies already issued land before the CTA can exit
-                for (int st = 0; st < 2; ++st) {
-                    if (last_k[st] >= 0) mbar_wait(&k_full[st], (last_k[st] >> 1) & 1, nullptr, 0);
-                    if (last_v[st] >= 0) mbar_wait(&v_full[st], (last_v[st] >> 1) & 1, nullptr, 0);
-                }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            g += it.nkt;
+        }
+        if (!ok && lane == 0) {
+            // let copies already issued land before the CTA can exit
+            for (int st = 0; st < 2; ++st) {
+                if (last_k[st] >= 0) mbar_wait(&k_full[st], (last_k[st] >> 1) & 1, nullptr, 0);
+                if (last_v[st] >= 0) mbar_wait(&v_full[st], (last_v[st] >> 1) & 1, nullptr, 0);
             }
         }
     } else if (warp == 1) {
@@ -215,9 +264,9 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
             constexpr uint32_t idS = idesc_bf16_f32(FA_ROWS, FA_KT);
             constexpr uint32_t idO = idesc_bf16_f32_bmn(FA_ROWS, FA_D);
             const uint32_t qa = smem_u32(Qs), pa = smem_u32(Ps);
-            auto issue_s = [&](int j) -> bool {
-                const int st = j & 1;
-                if (!mbar_wait(&k_full[st], (j >> 1) & 1, err, DERR_ATTN_MMA_WAIT)) return false;
+            auto issue_s = [&](int gg) -> bool {
+                const int st = gg & 1;
+                if (!mbar_wait(&k_full[st], (gg >> 1) & 1, err, DERR_ATTN_MMA_WAIT)) return false;
                 tc_fence_after();
                 const uint32_t ka = smem_u32(Ks + st * FA_TILE);
 #pragma unroll
@@ -230,24 +279,42 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
                 tc_commit(&s_full[st]);
                 return true;
             };
-            bool ok = issue_s(0);
-            if (ok && nkt > 1) ok = issue_s(1);
-            for (int j = 0; j < nkt && ok; ++j) {
-                const int st = j & 1;  // K/V stage, S accumulator and P buffer of tile j
-                if (!mbar_wait(&p_full[st], (j >> 1) & 1, err, DERR_ATTN_MMA_WAIT)) break;
-                if (!mbar_wait(&v_full[st], (j >> 1) & 1, err, DERR_ATTN_MMA_WAIT)) break;
+            bool ok = true;
+            int g = 0;
+            for (int ki = 0; ok; ++ki) {
+                const int k = item_of(ki);
+                if (k < 0) break;
+                const int nkt = describe(k).nkt;
+                if (ki > 0 && !mbar_wait(q_full, (ki - 1) & 1, err, DERR_ATTN_MMA_WAIT)) break;
                 tc_fence_after();
-                const uint32_t va = smem_u32(Vs + st * FA_TILE), pj = pa + st * FA_TILE;
+                ok = issue_s(g);
+                if (ok && nkt > 1) ok = issue_s(g + 1);
+                for (int j = 0; j < nkt && ok; ++j) {
+                    const int gg = g + j, st = gg & 1;  // K/V stage, S accumulator and P buffer
+                    if (!mbar_wait(&p_full[st], (gg >> 1) & 1, err, DERR_ATTN_MMA_WAIT)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!mbar_wait(&v_full[st], (gg >> 1) & 1, err, DERR_ATTN_MMA_WAIT)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t va = smem_u32(Vs + st * FA_TILE), pj = pa + st * FA_TILE;
 #pragma unroll
-                for (int kk = 0; kk < FA_KT / 16; ++kk) {
-                    // A = P: keys 16kk.. of the K-major P tile; B = V: the same 16 key rows,
-                    // all 128 dims (the second 64-dim half FA_HALF bytes on)
-                    tc_mma_f16(tmem_base + FA_TMEM_O, smem_desc_sw128(pj + (kk >> 2) * FA_HALF + (kk & 3) * 32),
-                               smem_desc_sw128_mn(va + kk * 2048, FA_HALF), idO, (j | kk) != 0);
+                    for (int kk = 0; kk < FA_KT / 16; ++kk) {
+                        // A = P: keys 16kk.. of the K-major P tile; B = V: the same 16 key rows,
+                        // all 128 dims (the second 64-dim half FA_HALF bytes on). The item's
+                        // first product overwrites O: the softmax threads read the previous
+                        // item's O before they released this P.
+                        tc_mma_f16(tmem_base + FA_TMEM_O, smem_desc_sw128(pj + (kk >> 2) * FA_HALF + (kk & 3) * 32),
+                                   smem_desc_sw128_mn(va + kk * 2048, FA_HALF), idO, (j | kk) != 0);
+                    }
+                    tc_commit(&v_empty[st]);
+                    tc_commit(&pv_done[st]);
+                    if (j + 2 < nkt) ok = issue_s(gg + 2);
                 }
-                tc_commit(&v_empty[st]);
-                tc_commit(&pv_done[st]);
-                if (j + 2 < nkt) ok = issue_s(j + 2);
+                g += nkt;
             }
             tc_commit(mma_done);  // arrives once every MMA issued above has completed
         }
@@ -255,120 +322,144 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         // ---------------- softmax (warps 2..9): two threads per row ----------------
         // Warps w and w+4 share TMEM lane quarter w % 4 (the rows); the first takes
         // keys 0..63 of each tile, the second keys 64..127. They agree on the row's
-        // maximum through shared memory and keep their own partial sums.
+        // maximum through shared memory and keep their own partial sums, added at
+        // the end through two free TMEM columns.
         const int q4 = warp & 3;             // the TMEM lane quarter this warp may access
         const int half = (warp - 2) >> 2;    // which 64 keys of a tile, and 64 dims of O
         const int r = q4 * 32 + lane;
-        const int rg = row0 + r;
-        const int t = rg / G, h = kvh * G + (rg - t * G);
-        const int prow = t < a.T ? p0 + t : -1;
         const uint32_t lane_base = tmem_base + ((uint32_t)(q4 * 32) << 16);
         const float sl2 = a.scale_log2;
-        float m_used = -INFINITY, l = 0.f;   // m_used in the log2 domain
         bool ok = true;
-        for (int j = 0; j < nkt; ++j) {
-            const int sb = j & 1;
-            if (ok && !mbar_wait(&s_full[sb], (j >> 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
-            tc_fence_after();
-            float s[64];
-            {
-                uint32_t u[2][32];
-#pragma unroll
-                for (int c = 0; c < 2; ++c) tc_ld_32x32b_x32(lane_base + sb * FA_KT + half * 64 + c * 32, u[c]);
-                tc_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 2; ++c)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(u[c][i]);
-            }
-            // raw maximum (the scale is positive), four independent chains
-            const int key0 = j * FA_KT + half * 64;
-            if (key0 + 63 > prow) {
-#pragma unroll
-                for (int i = 0; i < 64; ++i)
-                    if (key0 + i > prow) s[i] = -INFINITY;
-            }
-            float mx4[4] = {s[0], s[1], s[2], s[3]};
-#pragma unroll
-            for (int i = 4; i < 64; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], s[i]);
-            const __half mine = __float2half_ru(fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2);
-            red_max[sb][half][r] = mine;
-            named_bar_sync(1 + q4, 64);
-            const float mx = fmaxf(__half2float(mine), __half2float(red_max[sb][half ^ 1][r]));
-            const float m_new = fmaxf(m_used, mx);
-            const bool need = m_new > m_used + FA_RESCALE_LOG2;  // false while the row has seen no key
-            const float alpha = need ? ex2_approx(m_used - m_new) : 1.f;
-            // P buffer sb is free once PV of tile j-2 has completed
-            if (j >= 2 && ok && !mbar_wait(&pv_done[sb], ((j - 2) >> 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
-                // rescale this thread's 64 dims of O: PV of tile j-1 has completed, PV of
-                // tile j waits for this P
-                const int pb = (j - 1) & 1;
-                if (ok && !mbar_wait(&pv_done[pb], ((j - 1) >> 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
+        int g = 0;
+        for (int ki = 0;; ++ki) {
+            const int k = item_of(ki);
+            if (k < 0) break;
+            const FaItem it = describe(k);
+            const int rg = it.row0 + r;
+            const int t = rg / G, h = it.kvh * G + (rg - t * G);
+            const int prow = t < a.T ? it.p0 + t : -1;
+            float m_used = -INFINITY, l = 0.f;   // m_used in the log2 domain
+            for (int j = 0; j < it.nkt; ++j) {
+                const int gg = g + j, sb = gg & 1;
+                if (ok && !mbar_wait(&s_full[sb], (gg >> 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
                 tc_fence_after();
-#pragma unroll 1
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t u[32];
-                    tc_ld_32x32b_x32(lane_base + FA_TMEM_O + half * 64 + c * 32, u);
+                if (j == it.nkt - 1) {
+                    // the item's last S product is complete, so Q is free: stage the next
+                    // item's query rows now, and the MMA thread starts its S products
+                    // while this tile and the output of this item are finished
+                    const int kn = item_of(ki + 1);
+                    if (kn >= 0) {
+                        stage_q(describe(kn), threadIdx.x - 64, 256);
+                        fence_proxy_async();
+                        mbar_arrive(q_full);
+                    }
+                }
+                float s[64];
+                {
+                    uint32_t u[2][32];
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) tc_ld_32x32b_x32(lane_base + sb * FA_KT + half * 64 + c * 32, u[c]);
                     tc_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-                    tc_st_32x32b_x32(lane_base + FA_TMEM_O + half * 64 + c * 32, u);
-                }
-                tc_wait_st();
-            }
-            if (need) {
-                l *= alpha;
-                m_used = m_new;
-            }
-            const float muse = m_used == -INFINITY ? 0.f : m_used;
-            uint8_t* prow_s = Ps + sb * FA_TILE + half * FA_HALF + r * 128;
-            float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+                    for (int c = 0; c < 2; ++c)
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                float p[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    // a quarter of the exponentials on the FMA pipe
-                    const float x = fmaf(s[c * 8 + e], sl2, -muse);
-                    p[e] = e < 6 ? ex2_approx(x) : ex2_poly(x);
-                    sum4[e & 3] += p[e];
+                        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(u[c][i]);
                 }
-                const uint4 v = make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
-                                           pack_bf16x2(p[6], p[7]));
-                *reinterpret_cast<uint4*>(prow_s + ((c ^ (r & 7)) << 4)) = v;
-            }
-            l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-            fence_proxy_async();  // P is read by the tensor cores through the async proxy
-            tc_fence_before();
-            mbar_arrive(&p_full[sb]);
-        }
-        // PV of the last tile (and so every earlier one) has completed
-        if (ok && !mbar_wait(&pv_done[(nkt - 1) & 1], ((nkt - 1) >> 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
-        tc_fence_after();
-        // the row's sum is the two halves' sums (both taken against the same maximum),
-        // exchanged through the P buffers, which no MMA reads any more
-        float* red_l = reinterpret_cast<float*>(Ps);
-        red_l[half * FA_ROWS + r] = l;
-        named_bar_sync(1 + q4, 64);
-        l += red_l[(half ^ 1) * FA_ROWS + r];
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        __nv_bfloat16* dst = a.out + ((long long)(b * a.T + t) * a.H + h) * FA_D + half * 64;
+                // raw maximum (the scale is positive), four independent chains
+                const int key0 = j * FA_KT + half * 64;
+                if (key0 + 63 > prow) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        if (key0 + i > prow) s[i] = -INFINITY;
+                }
+                float mx4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+                for (int i = 4; i < 64; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], s[i]);
+                const __half mine = __float2half_ru(fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2);
+                red_max[sb][half][r] = mine;
+                named_bar_sync(1 + q4, 64);
+                const float mx = fmaxf(__half2float(mine), __half2float(red_max[sb][half ^ 1][r]));
+                const float m_new = fmaxf(m_used, mx);
+                const bool need = m_new > m_used + FA_RESCALE_LOG2;  // false while the row has seen no key
+                const float alpha = need ? ex2_approx(m_used - m_new) : 1.f;
+                // P buffer sb is free once PV of running tile gg-2 has completed
+                if (gg >= 2 && ok && !mbar_wait(&pv_done[sb], ((gg - 2) >> 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT))
+                    ok = false;
+                if (j > 0 && __any_sync(0xffffffffu, need)) {
+                    // rescale this thread's 64 dims of O: PV of the previous tile has
+                    // completed, PV of this one waits for this P
+                    const int pg = gg - 1;
+                    if (ok && !mbar_wait(&pv_done[pg & 1], (pg >> 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
+                    tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-            uint32_t u[32];
-            tc_ld_32x32b_x32(lane_base + FA_TMEM_O + half * 64 + c * 32, u);
-            tc_wait_ld();
-            if (prow >= 0) {
+                    for (int c = 0; c < 2; ++c) {
+                        uint32_t u[32];
+                        tc_ld_32x32b_x32(lane_base + FA_TMEM_O + half * 64 + c * 32, u);
+                        tc_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; i += 8) {
-                    const uint4 v = make_uint4(pack_bf16x2(__uint_as_float(u[i]) * inv, __uint_as_float(u[i + 1]) * inv),
-                                               pack_bf16x2(__uint_as_float(u[i + 2]) * inv, __uint_as_float(u[i + 3]) * inv),
-                                               pack_bf16x2(__uint_as_float(u[i + 4]) * inv, __uint_as_float(u[i + 5]) * inv),
-                                               pack_bf16x2(__uint_as_float(u[i + 6]) * inv, __uint_as_float(u[i + 7]) * inv));
-                    *reinterpret_cast<uint4*>(dst + c * 32 + i) = v;
+                        for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+                        tc_st_32x32b_x32(lane_base + FA_TMEM_O + half * 64 + c * 32, u);
+                    }
+                    tc_wait_st();
+                }
+                if (need) {
+                    l *= alpha;
+                    m_used = m_new;
+                }
+                const float muse = m_used == -INFINITY ? 0.f : m_used;
+                uint8_t* prow_s = Ps + sb * FA_TILE + half * FA_HALF + r * 128;
+                float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    float p[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        // a quarter of the exponentials on the FMA pipe
+                        const float x = fmaf(s[c * 8 + e], sl2, -muse);
+                        p[e] = e < 6 ? ex2_approx(x) : ex2_poly(x);
+                        sum4[e & 3] += p[e];
+                    }
+                    const uint4 v = make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]),
+                                               pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
+                    *reinterpret_cast<uint4*>(prow_s + ((c ^ (r & 7)) << 4)) = v;
+                }
+                l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+                fence_proxy_async();  // P is read by the tensor cores through the async proxy
+                tc_fence_before();
+                mbar_arrive(&p_full[sb]);
+            }
+            // PV of the item's last tile (and so every earlier one) has completed
+            const int gl = g + it.nkt - 1;
+            if (ok && !mbar_wait(&pv_done[gl & 1], (gl >> 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
+            tc_fence_after();
+            // the row's sum is the two halves' sums (both taken against the same
+            // maximum), exchanged through TMEM columns FA_TMEM_L + half of the row's lane
+            tc_st_x1(lane_base + FA_TMEM_L + half, __float_as_uint(l));
+            tc_wait_st();
+            tc_fence_before();
+            named_bar_sync(1 + q4, 64);
+            tc_fence_after();
+            l += __uint_as_float(tc_ld_x1(lane_base + FA_TMEM_L + (half ^ 1)));
+            tc_wait_ld();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            __nv_bfloat16* dst = a.out + ((long long)(it.b * a.T + t) * a.H + h) * FA_D + half * 64;
+#pragma unroll 1
+            for (int c = 0; c < 2; ++c) {
+                uint32_t u[32];
+                tc_ld_32x32b_x32(lane_base + FA_TMEM_O + half * 64 + c * 32, u);
+                tc_wait_ld();
+                if (prow >= 0) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        const uint4 v = make_uint4(pack_bf16x2(__uint_as_float(u[i]) * inv, __uint_as_float(u[i + 1]) * inv),
+                                                   pack_bf16x2(__uint_as_float(u[i + 2]) * inv, __uint_as_float(u[i + 3]) * inv),
+                                                   pack_bf16x2(__uint_as_float(u[i + 4]) * inv, __uint_as_float(u[i + 5]) * inv),
+                                                   pack_bf16x2(__uint_as_float(u[i + 6]) * inv, __uint_as_float(u[i + 7]) * inv));
+                        *reinterpret_cast<uint4*>(dst + c * 32 + i) = v;
+                    }
                 }
             }
+            g += it.nkt;
         }
     }
 
@@ -386,9 +477,11 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
 cudaError_t launch_attn_prefill(const AttnPrefillArgs& a, cudaStream_t s, bool pdl) {
     if (a.H % a.Hk != 0 || a.T < 1) return cudaErrorInvalidValue;
     const int G = a.H / a.Hk;
-    const long long nblk = (long long)((a.T * G + FA_ROWS - 1) / FA_ROWS) * a.B * a.Hk;
-    if (nblk > 0x7fffffffLL) return cudaErrorInvalidValue;
-    const dim3 grid((unsigned)nblk);
+    const long long items = (long long)((a.T * G + FA_ROWS - 1) / FA_ROWS) * a.B * a.Hk;
+    if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+    // persistent: one CTA per SM (the shared memory allows no second), never more CTAs than items
+    const int sms = current_num_sms();
+    const dim3 grid((unsigned)(items < sms ? items : sms));
     cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, FA_SMEM);
     if (e != cudaSuccess) return e;
     return launch_k(attn_prefill_kernel, grid, dim3(FA_THREADS), FA_SMEM, s, pdl, *a.tmK, *a.tmV, a);
