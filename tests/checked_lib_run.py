@@ -4,7 +4,8 @@ Loads the bounds-checking build of the library and runs small cases of every
 kernel family against the oracle with the device error word left at zero, then
 one out-of-range token id, which the checked embedding must report as
 LLM_ERR_DEVICE_BOUNDS without touching memory outside the table, after which
-the model keeps working.
+the model keeps working, and a prefill attention whose new tokens would run past
+the cache, reported the same way.
 """
 import os
 import sys
@@ -65,6 +66,18 @@ def ops():
     assert np.abs(O.f64(out.cpu()) - ref).max() <= bound
     out.zero_()
     L.llm_op_attention_decode_static(q.to(DEV), kc.to(DEV), vc.to(DEV), p, out)
+    L.llm_op_synchronize()
+    assert np.abs(O.f64(out.cpu()) - ref).max() <= bound
+    # new tokens that would run past the cache: the attention kernels read only
+    # inside it (their positions are clamped) and the checked build reports them
+    bad = torch.tensor([0, Smax - T + 1], dtype=torch.int32, device=DEV)
+    L.llm_op_attention_prefill(q.to(DEV), kc.to(DEV), vc.to(DEV), bad, out)
+    try:
+        L.llm_op_synchronize()
+        raise AssertionError("the checked build did not report the attention positions")
+    except L.LlmError as e:
+        assert e.code == L.LLM_ERR_DEVICE_BOUNDS and "attention" in str(e), (e.code, str(e))
+    L.llm_op_attention_prefill(q.to(DEV), kc.to(DEV), vc.to(DEV), p, out)
     L.llm_op_synchronize()
     assert np.abs(O.f64(out.cpu()) - ref).max() <= bound
 
