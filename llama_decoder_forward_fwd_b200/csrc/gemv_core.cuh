@@ -182,7 +182,7 @@ DEVI void gv_drain(const GvRing& r, long long issued, uint32_t* err, uint32_t co
 DEVI void gv_prologue(__nv_bfloat16* xs, const __nv_bfloat16* x, int ldx, int M, int K, int Kp, const NormIn& n,
                       int m0, float* rinv_s, float (*rred_s)[16], long long u0 = 0, long long u1 = -1, int nku = 1,
                       const __nv_bfloat16* xlo = nullptr) {
-    constexpr int XB = 8;  // 16-byte loads per thread per batch
+    constexpr int XB = 14;  // 16-byte loads per thread per batch: one batch covers the split rows of K = 14336
     // k blocks [kb0, kb1] (inclusive, wrapping past the row's end) of the range, or all
     const bool all_k = u1 < 0 || u1 - u0 >= nku;
     const int kb0 = all_k ? 0 : (int)(u0 % nku), kb1 = all_k ? 0 : (int)((u1 - 1) % nku);
