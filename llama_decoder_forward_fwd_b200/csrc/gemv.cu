@@ -119,12 +119,16 @@ __global__ void __launch_bounds__(GV_THREADS, gv_stages<EPI>() > 6 ? 1 : 2)
     X.ldx = a.ldx;
     X.M = a.M;
     X.K = a.K;
-    X.Kp = nku * GV_BK;
+    // the k blocks this CTA's units read: kb0, kb0 + 1, ... (mod nku)
+    const bool all_k = w.u1 - w.u0 >= nku || w.u1 <= w.u0;
+    X.kb0 = all_k ? 0 : (int)(w.u0 % nku);
+    X.nku = nku;
+    X.Kp = (all_k ? nku : (int)(w.u1 - w.u0)) * GV_BK;
     X.xlo = SPLIT ? a.x_lo : nullptr;
     X.MX = SPLIT ? 2 * a.M : a.M;
     X.xs = (long long)X.MX * X.Kp * 2 <= GV_XS_BYTES ? xs : nullptr;
-    gv_prologue(const_cast<__nv_bfloat16*>(X.xs), a.x, a.ldx, a.M, a.K, X.Kp, a.epi.norm, a.m0, rinv_s, rred_s, w.u0,
-                w.u1, nku, X.xlo);
+    gv_prologue(const_cast<__nv_bfloat16*>(X.xs), a.x, a.ldx, a.M, a.K, X.Kp, a.epi.norm, a.m0, rinv_s, rred_s, X.kb0,
+                nku, X.xlo);
     gv_consume<NB, EPI, SPLIT>(ring, w, X, a.N, a.m0, rinv_s, a.epi, a.ws, max_pieces, a.epi.err,
                                DERR_GEMV_CONSUMER_WAIT);
 }

@@ -170,27 +170,20 @@ DEVI void gv_drain(const GvRing& r, long long issued, uint32_t* err, uint32_t co
     }
 }
 
-// Consumers (256 threads), at the start of a projection: copy the M token rows
-// of x (row stride ldx, K % 8 == 0) into shared memory as [M][Kp], zero past K
-// (when xs is not null), and compute each row's RMSNorm scale from the partial
-// sums of h^2 left by the producer of the input (1 where the input is not
-// normed). Every load of the first batch is issued before any is used, so the
-// prologue costs about one memory round trip. Ends with a barrier of the consumers.
-// With a unit range [u0, u1) given (nku units per tile), only the 64-wide k
-// blocks those units read are copied: every CTA of a launch reads its own few
-// blocks instead of all of them reading the whole rows at once.
+// Consumers (256 threads), at the start of a projection: copy the token rows of x
+// (row stride ldx, K % 8 == 0) into shared memory (when xs is not null), and
+// compute each row's RMSNorm scale from the partial sums of h^2 left by the
+// producer of the input (1 where the input is not normed). Every load of the
+// first batch is issued before any is used, so the prologue costs about one
+// memory round trip. Ends with a barrier of the consumers.
+// Only the 64-wide k blocks the CTA's units read are copied, kb0, kb0 + 1, ...
+// (wrapping at nku, the blocks of a row), Kp / 64 of them: xs is [rows][Kp] with
+// slot s holding k block (kb0 + s) mod nku, zero past K. Every CTA of a launch
+// reads its own few blocks, and a range of many token rows still fits.
 DEVI void gv_prologue(__nv_bfloat16* xs, const __nv_bfloat16* x, int ldx, int M, int K, int Kp, const NormIn& n,
-                      int m0, float* rinv_s, float (*rred_s)[16], long long u0 = 0, long long u1 = -1, int nku = 1,
+                      int m0, float* rinv_s, float (*rred_s)[16], int kb0 = 0, int nku = 1 << 30,
                       const __nv_bfloat16* xlo = nullptr) {
     constexpr int XB = 14;  // 16-byte loads per thread per batch: one batch covers the split rows of K = 14336
-    // k blocks [kb0, kb1] (inclusive, wrapping past the row's end) of the range, or all
-    const bool all_k = u1 < 0 || u1 - u0 >= nku;
-    const int kb0 = all_k ? 0 : (int)(u0 % nku), kb1 = all_k ? 0 : (int)((u1 - 1) % nku);
-    auto needed = [&](int k) {
-        if (all_k) return true;
-        const int kb = k / GV_BK;
-        return kb0 <= kb1 ? (kb >= kb0 && kb <= kb1) : (kb >= kb0 || kb <= kb1);
-    };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // partial sums: the first part of each row, loads only
     float part[16];
@@ -209,9 +202,12 @@ DEVI void gv_prologue(__nv_bfloat16* xs, const __nv_bfloat16* x, int ldx, int M,
                 const int i = i0 + j * GV_CONSUMERS * 8;
                 v[j] = make_uint4(0, 0, 0, 0);
                 if (i < total) {
-                    const int r = i / Kp, k = i - r * Kp;
+                    const int r = i / Kp, ks = i - r * Kp;
+                    int kb = kb0 + ks / GV_BK;
+                    if (kb >= nku) kb -= nku;
+                    const int k = kb * GV_BK + (ks & (GV_BK - 1));
                     const __nv_bfloat16* src = xlo ? ((r & 1) ? xlo : x) + (size_t)(r >> 1) * ldx : x + (size_t)r * ldx;
-                    if (k < K && needed(k)) v[j] = __ldcg(reinterpret_cast<const uint4*>(src + k));
+                    if (k < K) v[j] = __ldcg(reinterpret_cast<const uint4*>(src + k));
                 }
             }
 #pragma unroll
@@ -244,8 +240,9 @@ DEVI void gv_prologue(__nv_bfloat16* xs, const __nv_bfloat16* x, int ldx, int M,
 // Token rows of one projection as the consumers see them.
 struct GvX {
     const __nv_bfloat16* x;  // [M][ldx] in global memory
-    int ldx, M, K, Kp;       // Kp: K padded to the unit width (the TMA box fills zeros past K)
+    int ldx, M, K, Kp;       // Kp: the row stride of xs, a whole number of 64-wide k blocks
     const __nv_bfloat16* xs; // [MX][Kp] copy in shared memory, or nullptr
+    int kb0 = 0, nku = 1 << 30;  // slot s of xs holds k block (kb0 + s) mod nku
     const __nv_bfloat16* xlo = nullptr;  // split activations: the remainders, [M][ldx]
     int MX = 0;                          // B-operand columns: M, or 2M when split
 };
@@ -512,7 +509,9 @@ DEVI bool gv_consume(GvRing& r, const GvWork& w, const GvX& X, int N, int m0, co
         for (int n = 0; n < NM; ++n) {
             const int mrow = g + 8 * n;
             if (X.xs) {
-                const uint32_t xp = xbase + (uint32_t)(mrow * X.Kp + k) * 2;
+                int slot = kx / GV_BK - X.kb0;
+                if (slot < 0) slot += X.nku;
+                const uint32_t xp = xbase + (uint32_t)(mrow * X.Kp + slot * GV_BK + t4 * 16) * 2;
                 xa[n] = z4;
                 xb[n] = z4;
                 if (mrow < MX) {
