@@ -63,25 +63,31 @@ DEVI void logits_finish(const Epi& e, int M, int ntiles, int* last_s) {
 // has in flight at its share of HBM bandwidth under load (measured at the
 // Llama-3-8B shape: 3.51 ms per decode token against 3.58 with 5 stages, 3.51 with
 // 7 or 9, 3.57 with 10); the lm_head, one long stream of 1 GB, keeps 10 stages
-// (163 against 172 us with 5).
-template <int EPI> constexpr int gv_stages() { return EPI == EPI_LOGITS ? 10 : 8; }
+// (163 against 172 us with 5). With 16 token columns (NB = 16: 5 to 16 tokens, or
+// their split parts) the residual projections (wo, and w2 with its long rows) keep 7
+// stages, so that 16 token rows of a CTA's k blocks of the 14336-wide FFN input (49
+// blocks at the Llama-3-8B shape) fit the staging buffer (batch 16: 7.26 -> 7.05 ms
+// per decode step); with one token (NB = 8) the deeper ring is the better use of the
+// shared memory.
+template <int NB, int EPI> constexpr bool gv_wide_xs() { return NB == 16 && EPI == EPI_RESID; }
+template <int NB, int EPI> constexpr int gv_stages() { return EPI == EPI_LOGITS ? 10 : gv_wide_xs<NB, EPI>() ? 7 : 8; }
 constexpr int GV_THREADS = GV_CONSUMERS + 32;   // 8 consumer warps + 1 producer warp
-constexpr int GV_XS_BYTES = 56 * 1024 + 256;    // token rows staged whole when they fit (one token's
-                                                // split rows of the 14336-wide FFN input)
-template <int EPI> constexpr int gv_smem() {
-    return 1024 + gv_stages<EPI>() * GV_UNIT_BYTES + GV_XS_BYTES + 2 * gv_stages<EPI>() * 8 + 64;
+// Token rows staged in shared memory when the CTA's k blocks of them fit.
+template <int NB, int EPI> constexpr int gv_xs_bytes() { return (gv_wide_xs<NB, EPI>() ? 98 : 56) * 1024 + 256; }
+template <int NB, int EPI> constexpr int gv_smem() {
+    return 1024 + gv_stages<NB, EPI>() * GV_UNIT_BYTES + gv_xs_bytes<NB, EPI>() + 2 * gv_stages<NB, EPI>() * 8 + 64;
 }
 
 template <int NB, int EPI, bool SPLIT>
-__global__ void __launch_bounds__(GV_THREADS, gv_stages<EPI>() > 6 ? 1 : 2)
+__global__ void __launch_bounds__(GV_THREADS, gv_stages<NB, EPI>() > 6 ? 1 : 2)
     gemv_bf16_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
                      const __grid_constant__ CUtensorMap tm2, const GemvArgs<__nv_bfloat16> a, int ntiles, int nku,
                      int max_pieces) {
-    constexpr int GV_STAGES = gv_stages<EPI>();
+    constexpr int GV_STAGES = gv_stages<NB, EPI>();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem + GV_STAGES * GV_UNIT_BYTES);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + GV_STAGES * GV_UNIT_BYTES + GV_XS_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + GV_STAGES * GV_UNIT_BYTES + gv_xs_bytes<NB, EPI>());
     __shared__ float rinv_s[16];
     __shared__ float rred_s[8][16];
     GvRing ring{smem, full, full + GV_STAGES, GV_STAGES, 0, 0u, 0};
@@ -126,7 +132,7 @@ __global__ void __launch_bounds__(GV_THREADS, gv_stages<EPI>() > 6 ? 1 : 2)
     X.Kp = (all_k ? nku : (int)(w.u1 - w.u0)) * GV_BK;
     X.xlo = SPLIT ? a.x_lo : nullptr;
     X.MX = SPLIT ? 2 * a.M : a.M;
-    X.xs = (long long)X.MX * X.Kp * 2 <= GV_XS_BYTES ? xs : nullptr;
+    X.xs = (long long)X.MX * X.Kp * 2 <= gv_xs_bytes<NB, EPI>() ? xs : nullptr;
     gv_prologue(const_cast<__nv_bfloat16*>(X.xs), a.x, a.ldx, a.M, a.K, X.Kp, a.epi.norm, a.m0, rinv_s, rred_s, X.kb0,
                 nku, X.xlo);
     gv_consume<NB, EPI, SPLIT>(ring, w, X, a.N, a.m0, rinv_s, a.epi, a.ws, max_pieces, a.epi.err,
@@ -265,7 +271,7 @@ static cudaError_t launch_bf16_e(const GemvArgs<__nv_bfloat16>& a, cudaStream_t 
     static bool smem_set = false;
     if (!smem_set) {
         cudaError_t e = cudaFuncSetAttribute(gemv_bf16_kernel<NB, EPI, SPLIT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, gv_smem<EPI>());
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, gv_smem<NB, EPI>());
         if (e != cudaSuccess) return e;
         smem_set = true;
     }
@@ -280,7 +286,7 @@ static cudaError_t launch_bf16_e(const GemvArgs<__nv_bfloat16>& a, cudaStream_t 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid);
     cfg.blockDim = dim3(GV_THREADS);
-    cfg.dynamicSmemBytes = gv_smem<EPI>();
+    cfg.dynamicSmemBytes = gv_smem<NB, EPI>();
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;
