@@ -13,9 +13,10 @@
 // kernel is persistent (one CTA per SM, TMEM allocated once): each CTA runs a
 // fixed sequence of items, longest causal rows first, and every role walks the
 // same sequence, so the barrier phases follow one running tile count. Keys go in
-// tiles of 128, d = 128. Ten warps:
-//   warp 0     TMA producer: K and V tiles (two 64-dim halves, 128-byte swizzle)
-//              from the KV cache into 2-stage rings, K and V on their own barriers;
+// tiles of 128, d = 128. Eleven warps:
+//   warps 0, 10  TMA producers, one thread each: K tiles (warp 0) and V tiles
+//              (warp 10), two 64-dim halves in the 128-byte swizzle, from the KV
+//              cache into 2-stage rings with their own barriers;
 //   warp 1     allocates 512 TMEM columns and issues tcgen05.mma from one thread:
 //              S = Q K^T (M = 128 rows, N = 128 keys, K = d) into one of two S
 //              accumulators, and O += P V (N = d, K = keys; V read MN-major, as it
@@ -43,7 +44,8 @@
 
 namespace lfw {
 
-constexpr int FA_THREADS = 320;
+constexpr int FA_THREADS = 352;
+constexpr int FA_V_WARP = 10;                   // the V producer
 constexpr int FA_ROWS = 128;
 constexpr int FA_KT = 128;                      // keys per tile
 constexpr int FA_D = 128;
@@ -64,17 +66,31 @@ DEVI float ex2_approx(float x) {
 }
 
 // 2^x on the FMA pipe, for a share of the elements so that the special-function
-// unit is not the only one computing exponentials: x = n + f with n the nearest
-// integer (added to the exponent field) and f in [-0.5, 0.5], 2^f by a cubic
-// fitted to minimise the relative error (at most 1.5e-4 in fp32 arithmetic, far
-// below the bf16 rounding P gets next). x is clamped at -126, so a masked score
-// gives 2^-126 instead of 0: nothing at the scale of the row's sum.
-DEVI float ex2_poly(float x) {
-    x = fmaxf(x, -126.f);
-    const float t = x + 12582912.f;       // 1.5 * 2^23: n lands in the low mantissa bits
-    const float f = x - (t - 12582912.f);
-    const float p = fmaf(fmaf(fmaf(0.05517166f, f, 0.24261114f), f, 0.69326097f), f, 0.99992806f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+// unit is not the only one computing exponentials, two values at a time with the
+// packed fp32 operations of sm_100 (one instruction per pair): x = n + f with n the
+// nearest integer (added to the exponent field) and f in [-0.5, 0.5], 2^f by a
+// cubic fitted to minimise the relative error (at most 1.5e-4 in fp32 arithmetic,
+// far below the bf16 rounding P gets next). x is clamped at -126, so a masked
+// score gives 2^-126 instead of 0: nothing at the scale of the row's sum.
+DEVI float2 ex2_poly2(float2 x) {
+    x.x = fmaxf(x.x, -126.f);
+    x.y = fmaxf(x.y, -126.f);
+    // 1.5 * 2^23: n lands in the low mantissa bits of t
+    const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+    const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);  // x - n, exact as a subtraction
+    float2 p = __ffma2_rn(make_float2(0.05517166f, 0.05517166f), f, make_float2(0.24261114f, 0.24261114f));
+    p = __ffma2_rn(p, f, make_float2(0.69326097f, 0.69326097f));
+    p = __ffma2_rn(p, f, make_float2(0.99992806f, 0.99992806f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+// max(a, b, c) in one instruction (three-input max of sm_100).
+DEVI float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 // tcgen05.st / tcgen05.ld of one 32-bit column of this thread's TMEM lane.
@@ -218,34 +234,34 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    if (warp == 0) {
-        // ---------------- producer: Q of each later item, K and V tiles ----------------
-        int last_k[2] = {it0.nkt > 0 ? 0 : -1, it0.nkt > 1 ? 1 : -1};  // last running tile loaded per stage
-        int last_v[2] = {last_k[0], last_k[1]};
+    if (warp == 0 || warp == FA_V_WARP) {
+        // ---------------- producers: K tiles (warp 0) and V tiles (the last warp) ----------------
+        // Each ring has its own thread, so a K tile is requested as soon as its stage
+        // is free (the S product two tiles back is complete), not after the V tile
+        // ahead of it, whose stage frees only when a PV product completes.
+        const bool is_v = warp == FA_V_WARP;
+        uint8_t* ring = is_v ? Vs : Ks;
+        const CUtensorMap* tm = is_v ? &tmV : &tmK;
+        uint64_t* full = is_v ? v_full : k_full;
+        uint64_t* empty = is_v ? v_empty : k_empty;
+        int last[2] = {it0.nkt > 0 ? 0 : -1, it0.nkt > 1 ? 1 : -1};  // last running tile loaded per stage
         bool ok = true;
         int g = 0;  // running tile index over this CTA's items
         for (int ki = 0; ok; ++ki) {
             const int k = item_of(ki);
             if (k < 0) break;
             const FaItem it = describe(k);
-            if (lane == 0) (void)LFW_CHECK(it.p0 >= 0 && it.p0 + a.T <= a.S_max, err, BC_ATTN_POS);
+            if (lane == 0 && !is_v) (void)LFW_CHECK(it.p0 >= 0 && it.p0 + a.T <= a.S_max, err, BC_ATTN_POS);
             const int j0 = ki == 0 ? min(2, it.nkt) : 0;
             if (lane == 0) {
                 for (int j = j0; j < it.nkt && ok; ++j) {
                     const int gg = g + j, st = gg & 1;
-                    const uint32_t ph = (gg >> 1) & 1;
-                    if (!mbar_wait(&k_empty[st], ph ^ 1u, err, DERR_ATTN_TMA_WAIT)) {
+                    if (!mbar_wait(&empty[st], ((gg >> 1) & 1) ^ 1u, err, DERR_ATTN_TMA_WAIT)) {
                         ok = false;
                         break;
                     }
-                    load_kv(Ks + st * FA_TILE, &tmK, &k_full[st], it.kv_row0, j);
-                    last_k[st] = gg;
-                    if (!mbar_wait(&v_empty[st], ph ^ 1u, err, DERR_ATTN_TMA_WAIT)) {
-                        ok = false;
-                        break;
-                    }
-                    load_kv(Vs + st * FA_TILE, &tmV, &v_full[st], it.kv_row0, j);
-                    last_v[st] = gg;
+                    load_kv(ring + st * FA_TILE, tm, &full[st], it.kv_row0, j);
+                    last[st] = gg;
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -253,10 +269,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         }
         if (!ok && lane == 0) {
             // let copies already issued land before the CTA can exit
-            for (int st = 0; st < 2; ++st) {
-                if (last_k[st] >= 0) mbar_wait(&k_full[st], (last_k[st] >> 1) & 1, nullptr, 0);
-                if (last_v[st] >= 0) mbar_wait(&v_full[st], (last_v[st] >> 1) & 1, nullptr, 0);
-            }
+            for (int st = 0; st < 2; ++st)
+                if (last[st] >= 0) mbar_wait(&full[st], (last[st] >> 1) & 1, nullptr, 0);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
@@ -374,8 +388,8 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
                 }
                 float mx4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-                for (int i = 4; i < 64; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], s[i]);
-                const __half mine = __float2half_ru(fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2);
+                for (int i = 4; i < 64; i += 2) mx4[(i >> 1) & 3] = fmax3(mx4[(i >> 1) & 3], s[i], s[i + 1]);
+                const __half mine = __float2half_ru(fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3])) * sl2);
                 red_max[sb][half][r] = mine;
                 named_bar_sync(1 + q4, 64);
                 const float mx = fmaxf(__half2float(mine), __half2float(red_max[sb][half ^ 1][r]));
@@ -397,7 +411,12 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
                         tc_ld_32x32b_x32(lane_base + FA_TMEM_O + half * 64 + c * 32, u);
                         tc_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+                        for (int i = 0; i < 32; i += 2) {
+                            const float2 o = __fmul2_rn(make_float2(__uint_as_float(u[i]), __uint_as_float(u[i + 1])),
+                                                        make_float2(alpha, alpha));
+                            u[i] = __float_as_uint(o.x);
+                            u[i + 1] = __float_as_uint(o.y);
+                        }
                         tc_st_32x32b_x32(lane_base + FA_TMEM_O + half * 64 + c * 32, u);
                     }
                     tc_wait_st();
@@ -408,22 +427,25 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
                 }
                 const float muse = m_used == -INFINITY ? 0.f : m_used;
                 uint8_t* prow_s = Ps + sb * FA_TILE + half * FA_HALF + r * 128;
-                float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+                // scores to exponents, exponentials and partial sums on pairs of keys
+                // (packed fp32: one instruction per pair)
+                const float2 sl2x2 = make_float2(sl2, sl2), nmx2 = make_float2(-muse, -muse);
+                float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    float p[8];
+                    float2 p[4];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 x = __ffma2_rn(make_float2(s[c * 8 + 2 * e], s[c * 8 + 2 * e + 1]), sl2x2, nmx2);
                         // a quarter of the exponentials on the FMA pipe
-                        const float x = fmaf(s[c * 8 + e], sl2, -muse);
-                        p[e] = e < 6 ? ex2_approx(x) : ex2_poly(x);
-                        sum4[e & 3] += p[e];
+                        p[e] = e < 3 ? make_float2(ex2_approx(x.x), ex2_approx(x.y)) : ex2_poly2(x);
+                        sum2[e & 1] = __fadd2_rn(sum2[e & 1], p[e]);
                     }
-                    const uint4 v = make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]),
-                                               pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7]));
+                    const uint4 v = make_uint4(pack_bf16x2(p[0].x, p[0].y), pack_bf16x2(p[1].x, p[1].y),
+                                               pack_bf16x2(p[2].x, p[2].y), pack_bf16x2(p[3].x, p[3].y));
                     *reinterpret_cast<uint4*>(prow_s + ((c ^ (r & 7)) << 4)) = v;
                 }
-                l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+                l += (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
                 fence_proxy_async();  // P is read by the tensor cores through the async proxy
                 tc_fence_before();
                 mbar_arrive(&p_full[sb]);
