@@ -19,20 +19,24 @@
 //              cache into 2-stage rings with their own barriers;
 //   warp 1     allocates 512 TMEM columns and issues tcgen05.mma from one thread:
 //              S = Q K^T (M = 128 rows, N = 128 keys, K = d) into one of two S
-//              accumulators, and O += P V (N = d, K = keys; V read MN-major, as it
-//              lies in the cache) into the O accumulator;
+//              accumulators, and O += P V (N = d, K = keys; P read from tensor
+//              memory, V from shared memory MN-major, as it lies in the cache) into
+//              the O accumulator;
 //   warps 2-9  softmax, two threads per row (its TMEM lane), 64 keys each:
 //              tcgen05.ld of the row of S, causal mask, the row's maximum (shared
 //              between the pair through shared memory), P = 2^(s - m) in the log2
-//              domain stored to shared memory in bf16 (two buffers) as the A operand
-//              of the PV product, partial sums; at the end tcgen05.ld of O / sum.
+//              domain stored with tcgen05.st to tensor memory in bf16 (two buffers)
+//              as the A operand of the PV product, partial sums; at the end
+//              tcgen05.ld of O / sum.
+// Keeping P in tensor memory leaves shared memory to the Q, K and V operands and the
+// TMA writes (160 KB a tile instead of 224 with P there).
 // The MMA thread issues S for tile j+2 as soon as P of tile j is written, and the
 // softmax of tile j+1 does not wait for PV of tile j (unless O must be rescaled),
 // so the tensor cores and the softmax warps work at the same time.
-// The softmax warps stage the next item's query rows as soon as the current item's
-// last S product is complete (in the swizzled layout, one memory round trip), so
-// the MMA thread starts the next item's S products while they finish the last
-// tile and write out O.
+// The softmax warps stage the next item's query rows (in the swizzled layout, one
+// memory round trip) once they have released P of the item's last tile, while that
+// PV product runs, so the MMA thread starts the next item's S products while they
+// write out O.
 // O is rescaled (tcgen05.ld, scale, tcgen05.st) only when a row's maximum grows
 // by more than 2^8 over the maximum its P values were taken against (the
 // conditional rescaling of FlashAttention-4): P stays below 256, exact in the
@@ -51,10 +55,10 @@ constexpr int FA_KT = 128;                      // keys per tile
 constexpr int FA_D = 128;
 constexpr int FA_HALF = 128 * 128;              // [128 rows][64 bf16]: 16 KB
 constexpr int FA_TILE = 2 * FA_HALF;            // a K, V, Q or P tile: 32 KB
-constexpr int FA_SMEM = 1024 + 7 * FA_TILE + 256;  // K, V (2 stages each), Q, P (2 buffers), barriers
-constexpr uint32_t FA_TMEM_COLS = 512;          // S (2 x 128 columns), O (128)
+constexpr int FA_SMEM = 1024 + 5 * FA_TILE + 256 + 1024;  // K, V (2 stages each), Q, barriers, row sums
+constexpr uint32_t FA_TMEM_COLS = 512;          // S (2 x 128 columns), O (128), P (2 x 64)
 constexpr uint32_t FA_TMEM_O = 256;
-constexpr uint32_t FA_TMEM_L = 384;             // two columns: the row sums of the pair's halves
+constexpr uint32_t FA_TMEM_P = 384;             // P in bf16, two keys per column, two buffers of 64
 constexpr float FA_RESCALE_LOG2 = 8.f;
 
 // 2^x by the special-function unit (ex2.approx, flush-to-zero): relative error of
@@ -93,14 +97,15 @@ DEVI float fmax3(float a, float b, float c) {
     return d;
 }
 
-// tcgen05.st / tcgen05.ld of one 32-bit column of this thread's TMEM lane.
-DEVI void tc_st_x1(uint32_t taddr, uint32_t v) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
-}
-DEVI uint32_t tc_ld_x1(uint32_t taddr) {
-    uint32_t v;
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v) : "r"(taddr) : "memory");
-    return v;
+// D (+)= A B with A in tensor memory (M = 128 rows in the lanes, two bf16 of a row
+// per 32-bit column along K) and B described in shared memory.
+DEVI void tc_mma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
 // A work item: the 128 rows of one (sequence, KV head) starting at row0.
@@ -114,12 +119,12 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
                         const AttnPrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // V stages sit below Q and P, so every operand read stays inside the allocation.
+    // V stages sit below Q, so every operand read stays inside the allocation.
     uint8_t* Ks = smem;                  // 2 stages
     uint8_t* Vs = smem + 2 * FA_TILE;    // 2 stages
     uint8_t* Qs = smem + 4 * FA_TILE;
-    uint8_t* Ps = smem + 5 * FA_TILE;    // 2 buffers
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 7 * FA_TILE);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 5 * FA_TILE);
+    float* lsum = reinterpret_cast<float*>(smem + 5 * FA_TILE + 256);  // [half][row]: the pair's row sums
     uint64_t* k_full = bars;
     uint64_t* k_empty = bars + 2;
     uint64_t* v_full = bars + 4;
@@ -277,7 +282,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16_f32(FA_ROWS, FA_KT);
             constexpr uint32_t idO = idesc_bf16_f32_bmn(FA_ROWS, FA_D);
-            const uint32_t qa = smem_u32(Qs), pa = smem_u32(Ps);
+            const uint32_t qa = smem_u32(Qs);
             auto issue_s = [&](int gg) -> bool {
                 const int st = gg & 1;
                 if (!mbar_wait(&k_full[st], (gg >> 1) & 1, err, DERR_ATTN_MMA_WAIT)) return false;
@@ -314,15 +319,15 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t va = smem_u32(Vs + st * FA_TILE), pj = pa + st * FA_TILE;
+                    const uint32_t va = smem_u32(Vs + st * FA_TILE), pj = tmem_base + FA_TMEM_P + st * 64;
 #pragma unroll
                     for (int kk = 0; kk < FA_KT / 16; ++kk) {
-                        // A = P: keys 16kk.. of the K-major P tile; B = V: the same 16 key rows,
-                        // all 128 dims (the second 64-dim half FA_HALF bytes on). The item's
-                        // first product overwrites O: the softmax threads read the previous
-                        // item's O before they released this P.
-                        tc_mma_f16(tmem_base + FA_TMEM_O, smem_desc_sw128(pj + (kk >> 2) * FA_HALF + (kk & 3) * 32),
-                                   smem_desc_sw128_mn(va + kk * 2048, FA_HALF), idO, (j | kk) != 0);
+                        // A = P from TMEM: keys 16kk.. are columns 8kk.. of the P buffer; B = V:
+                        // the same 16 key rows, all 128 dims (the second 64-dim half FA_HALF
+                        // bytes on). The item's first product overwrites O: the softmax
+                        // threads read the previous item's O before they released this P.
+                        tc_mma_f16_ta(tmem_base + FA_TMEM_O, pj + kk * 8, smem_desc_sw128_mn(va + kk * 2048, FA_HALF),
+                                      idO, (j | kk) != 0);
                     }
                     tc_commit(&v_empty[st]);
                     tc_commit(&pv_done[st]);
@@ -357,17 +362,6 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
                 const int gg = g + j, sb = gg & 1;
                 if (ok && !mbar_wait(&s_full[sb], (gg >> 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
                 tc_fence_after();
-                if (j == it.nkt - 1) {
-                    // the item's last S product is complete, so Q is free: stage the next
-                    // item's query rows now, and the MMA thread starts its S products
-                    // while this tile and the output of this item are finished
-                    const int kn = item_of(ki + 1);
-                    if (kn >= 0) {
-                        stage_q(describe(kn), threadIdx.x - 64, 256);
-                        fence_proxy_async();
-                        mbar_arrive(q_full);
-                    }
-                }
                 float s[64];
                 {
                     uint32_t u[2][32];
@@ -426,11 +420,11 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
                     m_used = m_new;
                 }
                 const float muse = m_used == -INFINITY ? 0.f : m_used;
-                uint8_t* prow_s = Ps + sb * FA_TILE + half * FA_HALF + r * 128;
                 // scores to exponents, exponentials and partial sums on pairs of keys
                 // (packed fp32: one instruction per pair)
                 const float2 sl2x2 = make_float2(sl2, sl2), nmx2 = make_float2(-muse, -muse);
                 float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                uint32_t pw[32];  // this thread's 64 keys of P in bf16 pairs: TMEM columns of its lane
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     float2 p[4];
@@ -441,28 +435,38 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
                         p[e] = e < 3 ? make_float2(ex2_approx(x.x), ex2_approx(x.y)) : ex2_poly2(x);
                         sum2[e & 1] = __fadd2_rn(sum2[e & 1], p[e]);
                     }
-                    const uint4 v = make_uint4(pack_bf16x2(p[0].x, p[0].y), pack_bf16x2(p[1].x, p[1].y),
-                                               pack_bf16x2(p[2].x, p[2].y), pack_bf16x2(p[3].x, p[3].y));
-                    *reinterpret_cast<uint4*>(prow_s + ((c ^ (r & 7)) << 4)) = v;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) pw[c * 4 + e] = pack_bf16x2(p[e].x, p[e].y);
                 }
                 l += (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
-                fence_proxy_async();  // P is read by the tensor cores through the async proxy
+                // P buffer sb in TMEM: the A operand of the PV product (row = lane, key
+                // pairs along the columns)
+                tc_st_32x32b_x32(lane_base + FA_TMEM_P + sb * 64 + half * 32, pw);
+                tc_wait_st();
                 tc_fence_before();
                 mbar_arrive(&p_full[sb]);
+            }
+            {
+                // the item's last S product is complete, so Q is free: stage the next
+                // item's query rows while PV of the last tile runs; the MMA thread then
+                // starts the next item's S products while this item's output is written
+                const int kn = item_of(ki + 1);
+                if (kn >= 0) {
+                    stage_q(describe(kn), threadIdx.x - 64, 256);
+                    fence_proxy_async();
+                    mbar_arrive(q_full);
+                }
             }
             // PV of the item's last tile (and so every earlier one) has completed
             const int gl = g + it.nkt - 1;
             if (ok && !mbar_wait(&pv_done[gl & 1], (gl >> 1) & 1, err, DERR_ATTN_SOFTMAX_WAIT)) ok = false;
             tc_fence_after();
             // the row's sum is the two halves' sums (both taken against the same
-            // maximum), exchanged through TMEM columns FA_TMEM_L + half of the row's lane
-            tc_st_x1(lane_base + FA_TMEM_L + half, __float_as_uint(l));
-            tc_wait_st();
-            tc_fence_before();
+            // maximum), exchanged through shared memory (the partner reads the value
+            // before the next tile's barrier, so one slot per half suffices)
+            lsum[half * FA_ROWS + r] = l;
             named_bar_sync(1 + q4, 64);
-            tc_fence_after();
-            l += __uint_as_float(tc_ld_x1(lane_base + FA_TMEM_L + (half ^ 1)));
-            tc_wait_ld();
+            l += lsum[(half ^ 1) * FA_ROWS + r];
             const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16* dst = a.out + ((long long)(it.b * a.T + t) * a.H + h) * FA_D + half * 64;
 #pragma unroll 1
