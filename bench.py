@@ -35,12 +35,20 @@ METRIC = "decode & prefill tokens/s at Llama-3-8B shape, 1 B200; % of HBM/tensor
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def load_peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+def load_peaks(path=None):
+    """The roofline denominators: the measured HBM copy bandwidth (GB/s) and bf16 GEMM
+    rates (TF/s) when MEASURED_PEAKS.json holds them as numbers, else the fallback."""
+    p = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
-        d = json.load(open(p))
-        return d, "measured"
-    return PEAKS_FALLBACK, "fallback"
+        try:
+            d = json.load(open(p))
+            peaks = {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops")}
+            peaks["bf16_tflops_sustained"] = float(d.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+            if min(peaks.values()) > 0:
+                return peaks, "measured"
+        except (OSError, ValueError, TypeError, KeyError, AttributeError):
+            pass
+    return dict(PEAKS_FALLBACK), "fallback"
 
 
 # ---------------------------------------------------------------- algorithmic work

@@ -66,3 +66,22 @@ def test_batched_workload_bytes_scale_the_cache_by_the_batch():
 
 def test_replica_throughput_counts_every_rank():
     assert bench.replica_throughput(4, 5, 2304, 2.0) == pytest.approx(4 * 5 * 2304 / 2.0)
+
+
+def test_peaks_come_from_the_measured_file_and_fall_back_when_it_is_unusable(tmp_path):
+    import json
+
+    p = tmp_path / "peaks.json"
+    p.write_text(json.dumps({"hbm_gbs": 6547.5, "bf16_tflops": 1674.6, "bf16_tflops_sustained": 1363.4,
+                             "clocks": {"sm_mhz": 1965}}))
+    peaks, src = bench.load_peaks(str(p))
+    assert src == "measured"
+    assert peaks == {"hbm_gbs": 6547.5, "bf16_tflops": 1674.6, "bf16_tflops_sustained": 1363.4}
+    p.write_text(json.dumps({"hbm_gbs": 6547.5, "bf16_tflops": 1674.6}))
+    assert bench.load_peaks(str(p))[0]["bf16_tflops_sustained"] == 1674.6
+    for bad in ('{"hbm_gbs": 6547.5}', '{"hbm_gbs": "n/a", "bf16_tflops": 1}', "[1, 2]", "not json",
+                '{"hbm_gbs": 0, "bf16_tflops": 1674.6}'):
+        p.write_text(bad)
+        peaks, src = bench.load_peaks(str(p))
+        assert src == "fallback" and peaks == bench.PEAKS_FALLBACK
+    assert bench.load_peaks(str(tmp_path / "absent.json"))[1] == "fallback"
